@@ -1,0 +1,237 @@
+// api.cu -- the C ABI: argument checks, workspace carving, launches.
+//
+// Every entry point checks its arguments on the host first and launches nothing
+// when a check fails.  The checks mirror the pages' own: "minimax_h3_nvfp4_decoder"
+// -- NVFP4DecoderLinear.__init__ (in_features % 16, in_features % rotation_group)
+// and from_packed (packed weight shape); "convert_minimax_h3_text_encoder_nvfp4.py"
+// -- quantize_language_linear (exact packed and scale shapes).
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+// Per-device asynchronous status word (see nvfp4_last_device_status).
+__device__ int g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+int* g_status_ptr[kMaxDevices];
+std::mutex g_mu;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool valid_group(int g) { return g == 0 || g == 16 || g == 32 || g == 64 || g == 128; }
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Workspace carving for nvfp4_linear: packed x | scales | {gsf_x, alpha} | partials.
+struct LinearWs {
+    size_t packed, sf, scalars, partials, total;
+};
+
+LinearWs linear_ws(int64_t M, int64_t K) {
+    LinearWs w;
+    w.packed = 0;
+    w.sf = align256((size_t)M * (size_t)K / 2);
+    w.scalars = w.sf + align256(nvfp4_scale_bytes(M, K));
+    w.partials = w.scalars + 256;
+    w.total = w.partials + align256(kQuantWorkspace);
+    return w;
+}
+
+}  // namespace
+
+nvfp4_status device_info(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (g_dev[dev].device != dev) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+        g_dev[dev].sms = prop.multiProcessorCount;
+        g_dev[dev].major = prop.major;
+        g_dev[dev].minor = prop.minor;
+        g_dev[dev].device = dev;
+    }
+    *out = g_dev[dev];
+    if (out->major != 10 || out->minor != 0) return NVFP4_ERR_DEVICE;
+    return NVFP4_OK;
+}
+
+nvfp4_status status_word(int** dev_ptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return NVFP4_ERR_CUDA;
+        g_status_ptr[dev] = static_cast<int*>(p);
+    }
+    *dev_ptr = g_status_ptr[dev];
+    return NVFP4_OK;
+}
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" {
+
+const char* nvfp4_status_string(int s) {
+    switch (s) {
+        case NVFP4_OK: return "NVFP4_OK";
+        case NVFP4_ERR_INVALID_ARG: return "NVFP4_ERR_INVALID_ARG";
+        case NVFP4_ERR_SHAPE: return "NVFP4_ERR_SHAPE";
+        case NVFP4_ERR_ALIGN: return "NVFP4_ERR_ALIGN";
+        case NVFP4_ERR_WORKSPACE: return "NVFP4_ERR_WORKSPACE";
+        case NVFP4_ERR_DEVICE: return "NVFP4_ERR_DEVICE";
+        case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
+        case NVFP4_ERR_TIMEOUT: return "NVFP4_ERR_TIMEOUT";
+        default: return "NVFP4_ERR_UNKNOWN";
+    }
+}
+
+int nvfp4_abi_version(void) { return 1; }
+
+size_t nvfp4_scale_bytes(int64_t rows, int64_t K) {
+    if (rows <= 0 || K <= 0) return 0;
+    return (size_t)((rows + 127) / 128 * 128) * (size_t)((K / 16 + 3) / 4 * 4);
+}
+
+size_t nvfp4_packed_bytes(int64_t rows, int64_t K) {
+    if (rows <= 0 || K <= 0) return 0;
+    return (size_t)rows * (size_t)(K / 2);
+}
+
+nvfp4_status hadamard_rotate(const void* x, void* y, int64_t rows, int64_t K, int group,
+                             void* stream) {
+    if (!x || !y || rows < 0 || group == 0 || !valid_group(group)) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % group) return NVFP4_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(y, 16)) return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (rows == 0) return NVFP4_OK;
+    return launch_rotate(x, y, rows, K, group, static_cast<cudaStream_t>(stream));
+}
+
+size_t nvfp4_quantize_workspace_bytes(void) { return kQuantWorkspace; }
+
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int group,
+                            const float* gsf_in, float* gsf_out, uint8_t* packed, uint8_t* sf,
+                            void* workspace, size_t ws_bytes, void* stream) {
+    if (!x || !packed || !sf || rows < 0 || !valid_group(group)) return NVFP4_ERR_INVALID_ARG;
+    if (!gsf_in && !gsf_out) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 16 || (group && K % group)) return NVFP4_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(sf, 16)) return NVFP4_ERR_ALIGN;
+    if ((gsf_in && !aligned(gsf_in, 4)) || (gsf_out && !aligned(gsf_out, 4)))
+        return NVFP4_ERR_ALIGN;
+    if (!gsf_in) {
+        if (!workspace || ws_bytes < kQuantWorkspace) return NVFP4_ERR_WORKSPACE;
+        if (!aligned(workspace, 16)) return NVFP4_ERR_ALIGN;
+    }
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (rows == 0) return NVFP4_OK;
+    return launch_quantize(x, rows, K, group, gsf_in, gsf_out, packed, sf,
+                           static_cast<float*>(workspace), nullptr, nullptr,
+                           static_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                        const uint8_t* sfb, const float* alpha, const void* bias, void* y,
+                        int64_t M, int64_t N, int64_t K, void* stream) {
+    if (!a || !sfa || !b || !sfb || !alpha || !y || M < 0 || N < 0) return NVFP4_ERR_INVALID_ARG;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 64 || K >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+    if (!aligned(a, 16) || !aligned(sfa, 16) || !aligned(b, 16) || !aligned(sfb, 16) ||
+        !aligned(y, 16) || !aligned(alpha, 4) || (bias && !aligned(bias, 16)))
+        return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    return launch_gemm(a, sfa, b, sfb, alpha, bias, y, M, N, K, static_cast<cudaStream_t>(stream));
+}
+
+size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K) {
+    if (M < 0 || K <= 0) return 0;
+    return linear_ws(M, K).total;
+}
+
+nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w_packed,
+                          const uint8_t* w_sf, const float* gsf_w, int64_t N, const void* bias,
+                          const float* gsf_x, int group, void* workspace, size_t ws_bytes,
+                          void* y, void* stream) {
+    if (!x || !w_packed || !w_sf || !gsf_w || !y || M < 0 || N < 0 || !valid_group(group))
+        return NVFP4_ERR_INVALID_ARG;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 64 || (group && K % group) || K >= (int64_t(1) << 31))
+        return NVFP4_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(w_packed, 16) || !aligned(w_sf, 16) || !aligned(y, 16) ||
+        !aligned(gsf_w, 4) || (gsf_x && !aligned(gsf_x, 4)) || (bias && !aligned(bias, 16)))
+        return NVFP4_ERR_ALIGN;
+    const LinearWs ws = linear_ws(M, K);
+    if (!workspace || ws_bytes < ws.total) return NVFP4_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return NVFP4_OK;
+
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    uint8_t* xp = base + ws.packed;
+    uint8_t* xsf = base + ws.sf;
+    float* scalars = reinterpret_cast<float*>(base + ws.scalars);
+    float* partials = reinterpret_cast<float*>(base + ws.partials);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_quantize(x, M, K, group, gsf_x, &scalars[0], xp, xsf, partials, gsf_w, &scalars[1],
+                         s);
+    if (st != NVFP4_OK) return st;
+    return launch_gemm(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s);
+}
+
+nvfp4_status nvfp4_last_device_status(void* stream, int* status) {
+    if (!status) return NVFP4_ERR_INVALID_ARG;
+    int* dev_ptr = nullptr;
+    nvfp4_status st = status_word(&dev_ptr);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int host = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (cudaMemcpyAsync(&host, dev_ptr, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    if (cudaMemsetAsync(dev_ptr, 0, sizeof(int), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    *status = host;
+    return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_debug_cvt_sweep(uint32_t first, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
+                                   void* stream) {
+    if (!e2m1 || !e4m3 || n < 0 || n > (int64_t(1) << 32)) return NVFP4_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (n == 0) return NVFP4_OK;
+    return launch_cvt_sweep(first, n, e2m1, e4m3, static_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status nvfp4_debug_wait_timeout(int64_t budget_us, void* stream) {
+    if (budget_us < 1 || budget_us > 2000000) return NVFP4_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    return launch_wait_timeout(budget_us, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

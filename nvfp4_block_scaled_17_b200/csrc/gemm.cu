@@ -1,0 +1,341 @@
+// gemm.cu -- block-scaled FP4 x FP4 GEMM on the sm_100a tensor cores.
+//
+// Pages: "minimax_h3_nvfp4_decoder" -- nvfp4_linear_inference: mm_fp4 over the
+// packed activation and weight with their E4M3 block scales (block_size 16, 128x4
+// layout), alpha = 1/(global_sf_x * global_sf_w) applied to the product, bf16
+// output, then the bias added.  Here alpha and the bias are fused into the
+// epilogue: y = bf16(fp32(alpha * acc) + bias).
+//
+// Design (one CTA per SM, persistent over 128 x 256 output tiles):
+//   warp 0      TMA producer: per 256-wide K step, a 128 x 128-byte A box and a
+//               256 x 128-byte B box (128-byte swizzle), plus the matching 512-byte
+//               chunks of the 128x4 scale layout with plain bulk copies (the layout
+//               already is the tensor-memory copy order, so no reshuffle is needed).
+//   warp 1      MMA issuer (one lane): tcgen05.cp of the scale chunks into tensor
+//               memory, then tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64)
+//               four times per stage, accumulating in tensor memory; tcgen05.commit
+//               releases the stage and, at the end of a tile, hands the accumulator to
+//               the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quadrant, alpha, bias, bf16,
+//               stores.
+// Every wait is bounded (globaltimer); on expiry the kernel records
+// NVFP4_ERR_TIMEOUT, drains its own copies and MMAs, frees tensor memory and exits.
+// No load uses cluster multicast.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <cudaTypedefs.h>
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr int BM = 128;                 // rows of A per tile (= tensor-memory lanes)
+constexpr int BN = 256;                 // rows of B per tile (= accumulator columns)
+constexpr int BKB = 128;                // bytes of packed K per stage (256 values)
+constexpr int STAGES = 4;
+constexpr int SMEM_A = BM * BKB;        // 16 KiB
+constexpr int SMEM_B = BN * BKB;        // 32 KiB
+constexpr int SMEM_SFA = 4 * 512;       // four K=64 scale chunks for 128 rows
+constexpr int SMEM_SFB = 8 * 512;       // the same for 256 rows (two 128-row tiles)
+constexpr int TMEM_COLS = 512;
+constexpr int TMEM_SFA = 256;           // 4 chunks x 4 columns
+constexpr int TMEM_SFB = 272;           // 4 chunks x 8 columns
+constexpr int THREADS = 192;
+constexpr int SMEM_BYTES = 1024 + STAGES * (SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB) + 256;
+
+// Instruction descriptor: E2M1 x E2M1 (format 1), both K-major, UE4M3 scales,
+// N = 256, M = 128, dense K = 64.
+constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                           ((uint32_t)(BM >> 4) << 24);
+
+struct GemmParams {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const float* alpha;
+    const uint16_t* bias;      // bf16 [N] or null
+    uint16_t* y;               // bf16 [M, N]
+    int M, N;
+    int m_blocks, n_blocks;
+    int k_tiles;               // ceil(K / 256)
+    int kchunks;               // K / 64: scale chunks per 128-row tile
+    int sf_row_tiles_b;        // ceil(N / 128)
+    int* status;
+    uint64_t budget_ns;
+};
+
+__device__ __forceinline__ uint16_t bf16_bits_rn(float v) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + STAGES * SMEM_A;
+    uint8_t* sSFA = sB + STAGES * SMEM_B;
+    uint8_t* sSFB = sSFA + STAGES * SMEM_SFA;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SMEM_SFB);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* drain = acc_empty + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 4);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    const int num_tiles = p.m_blocks * p.n_blocks;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tensormap(&tmA);
+            prefetch_tensormap(&tmB);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_phase = 0;   // per-stage bit masks
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                const int m_blk = tile % p.m_blocks;
+                const int n_blk = tile / p.m_blocks;
+                const int sfb_tiles = (2 * n_blk + 1 < p.sf_row_tiles_b) ? 2 : 1;
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status,
+                                           p.budget_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const int steps = min(4, p.kchunks - 4 * kt);
+                    const uint32_t sf_bytes = (uint32_t)steps * 512u;
+                    mbar_arrive_expect_tx(&full[stage], SMEM_A + SMEM_B + sf_bytes * (1 + sfb_tiles));
+                    tma_load_2d(sA + stage * SMEM_A, &tmA, &full[stage], kt * BKB, m_blk * BM);
+                    tma_load_2d(sB + stage * SMEM_B, &tmB, &full[stage], kt * BKB, n_blk * BN);
+                    bulk_load(sSFA + stage * SMEM_SFA,
+                              p.sfa + ((size_t)m_blk * p.kchunks + 4 * kt) * 512, sf_bytes,
+                              &full[stage]);
+                    for (int t = 0; t < sfb_tiles; ++t)
+                        bulk_load(sSFB + stage * SMEM_SFB + t * 2048,
+                                  p.sfb + ((size_t)(2 * n_blk + t) * p.kchunks + 4 * kt) * 512,
+                                  sf_bytes, &full[stage]);
+                    issued |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            // Every fill this thread started must land before the block can exit.
+            for (int s = 0; s < STAGES; ++s)
+                if (issued & (1u << s)) {
+                    volatile int no_abort = 0;
+                    mbar_wait_bounded(&full[s], (issued_phase >> s) & 1, &no_abort, p.status,
+                                      p.budget_ns);
+                }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                const int n_blk = tile / p.m_blocks;
+                (void)n_blk;
+                if (!mbar_wait_bounded(acc_empty, acc_phase ^ 1, abort_flag, p.status,
+                                       p.budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status,
+                                           p.budget_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int steps = min(4, p.kchunks - 4 * kt);
+                    const uint32_t a0 = smem_u32(sA + stage * SMEM_A);
+                    const uint32_t b0 = smem_u32(sB + stage * SMEM_B);
+                    const uint32_t sfa0 = smem_u32(sSFA + stage * SMEM_SFA);
+                    const uint32_t sfb0 = smem_u32(sSFB + stage * SMEM_SFB);
+                    for (int kk = 0; kk < steps; ++kk) {
+                        tc_copy_sf(tmem + TMEM_SFA + 4 * kk, sdesc_sf(sfa0 + 512 * kk));
+                        tc_copy_sf(tmem + TMEM_SFB + 8 * kk, sdesc_sf(sfb0 + 512 * kk));
+                        tc_copy_sf(tmem + TMEM_SFB + 8 * kk + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
+                    }
+                    for (int kk = 0; kk < steps; ++kk) {
+                        mma_nvf4(tmem, sdesc_kmajor_sw128(a0 + 32 * kk),
+                                 sdesc_kmajor_sw128(b0 + 32 * kk), IDESC, tmem + TMEM_SFA + 4 * kk,
+                                 tmem + TMEM_SFB + 8 * kk, (kt | kk) != 0);
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(acc_full);
+                acc_phase ^= 1;
+            }
+            // Wait until every tensor-core operation this thread issued has finished.
+            tc_commit(drain);
+            volatile int no_abort = 0;
+            mbar_wait_bounded(drain, 0, &no_abort, p.status, p.budget_ns);
+        }
+        __syncwarp();
+    } else {
+        // epilogue: warp w reads tensor-memory lanes 32*(w%4) .. 32*(w%4)+31
+        const int quad = warp & 3;
+        const float alpha = *p.alpha;
+        const bool vec_ok = (p.N % 8) == 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const int m_blk = tile % p.m_blocks;
+            const int n_blk = tile / p.m_blocks;
+            if (!mbar_wait_bounded(acc_full, acc_phase, abort_flag, p.status, p.budget_ns)) break;
+            tc_fence_after();
+            const int row = m_blk * BM + quad * 32 + lane;
+            uint16_t* yrow = p.y + (size_t)row * p.N;
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                const int n0 = n_blk * BN + c0;
+                if (n0 >= p.N) break;   // warp-uniform
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, r);
+                tmem_ld_wait();
+                uint32_t packed[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    float v0 = __fmul_rn(alpha, __uint_as_float(r[j]));
+                    float v1 = __fmul_rn(alpha, __uint_as_float(r[j + 1]));
+                    if (p.bias) {
+                        const int na = min(n0 + j, p.N - 1), nb = min(n0 + j + 1, p.N - 1);
+                        v0 = __fadd_rn(v0, __uint_as_float((uint32_t)p.bias[na] << 16));
+                        v1 = __fadd_rn(v1, __uint_as_float((uint32_t)p.bias[nb] << 16));
+                    }
+                    packed[j / 2] = (uint32_t)bf16_bits_rn(v0) | ((uint32_t)bf16_bits_rn(v1) << 16);
+                }
+                if (row < p.M) {
+                    if (vec_ok && n0 + 32 <= p.N) {
+                        uint4* d = reinterpret_cast<uint4*>(yrow + n0);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            d[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+                                              packed[4 * q + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (n0 + j < p.N) yrow[n0 + j] = (uint16_t)(packed[j / 2] >> (16 * (j & 1)));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+            acc_phase ^= 1;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D uint8 view [rows, row_bytes] with a [box_rows, 128-byte] box, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)BKB, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                         const uint8_t* sfb, const float* alpha, const void* bias, void* y,
+                         int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    int* status = nullptr;
+    if ((st = status_word(&status)) != NVFP4_OK) return st;
+
+    CUtensorMap mapA, mapB;
+    if (!make_map(&mapA, a, M, K / 2, BM) || !make_map(&mapB, b, N, K / 2, BN))
+        return NVFP4_ERR_CUDA;
+
+    static bool attr_set[64] = {false};
+    if (!attr_set[dev.device & 63]) {
+        if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_BYTES) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        attr_set[dev.device & 63] = true;
+    }
+
+    GemmParams p{};
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.alpha = alpha;
+    p.bias = static_cast<const uint16_t*>(bias);
+    p.y = static_cast<uint16_t*>(y);
+    p.M = (int)M;
+    p.N = (int)N;
+    p.m_blocks = (int)((M + BM - 1) / BM);
+    p.n_blocks = (int)((N + BN - 1) / BN);
+    p.k_tiles = (int)((K + 255) / 256);
+    p.kchunks = (int)(K / 64);
+    p.sf_row_tiles_b = (int)((N + 127) / 128);
+    p.status = status;
+    p.budget_ns = 4000000000ull;   // 4 s
+
+    const int tiles = p.m_blocks * p.n_blocks;
+    const int grid = tiles < dev.sms ? tiles : dev.sms;
+    gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(mapA, mapB, p);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,44 @@
+// kernels.h -- host-side launchers shared between the translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nvfp4.h"
+
+namespace nvfp4 {
+
+// Cached per-device facts (multiprocessor count, compute capability).
+struct DeviceInfo {
+    int device = -1;
+    int sms = 0;
+    int major = 0, minor = 0;
+};
+nvfp4_status device_info(DeviceInfo* out);
+
+// Rotation scale rn(1/sqrt(g)) for g in {16, 32, 64, 128}.
+float hadamard_scale(int g);
+
+// Quantizer: [rotate] -> [amax pass] -> encode pass.  `partials` (kMaxPartials
+// floats) is required when gsf_in == nullptr.  When gsf_w and alpha_out are
+// given the encode pass also writes alpha = rn(1 / rn(gsf * gsf_w)).
+nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
+                             const float* gsf_in, float* gsf_out, uint8_t* packed, uint8_t* sf,
+                             float* partials, const float* gsf_w, float* alpha_out,
+                             cudaStream_t stream);
+
+nvfp4_status launch_rotate(const void* x, void* y, int64_t rows, int64_t K, int group,
+                           cudaStream_t stream);
+
+nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                         const uint8_t* sfb, const float* alpha, const void* bias, void* y,
+                         int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+
+nvfp4_status launch_cvt_sweep(uint32_t first, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
+                              cudaStream_t stream);
+nvfp4_status launch_wait_timeout(int64_t budget_us, cudaStream_t stream);
+
+// The per-device asynchronous status word (device address for the current device).
+nvfp4_status status_word(int** dev_ptr);
+
+}  // namespace nvfp4

@@ -1,0 +1,128 @@
+"""GPU parity of the block-scaled FP4 GEMM and of the whole linear against the
+fp64 oracle over the same dequantized operands, through the C ABI.
+
+Bound: relative Frobenius error <= 2e-3 and max-abs error <= 1e-2 * rms(y) (+ one
+bf16 ulp of the reference for the bf16 output).  Pages: "minimax_h3_nvfp4_decoder"
+-- nvfp4_linear_inference (mm_fp4 with alpha = 1/(gsf_x*gsf_w), then the bias);
+"convert_minimax_h3_text_encoder_nvfp4.py" -- probe_relative_error (W4A4 error about
+0.13 on random N(0,1) rows with a unit activation scale).
+"""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_17_b200 as nv
+from nvfp4_block_scaled_17_b200 import workloads as W
+from gpu_util import assert_gemm_close, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def t(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def sample_rows(M: int, n: int, seed: int = 0) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    pick = {0, M - 1, min(127, M - 1), min(128, M - 1)}
+    pick |= set(rng.integers(0, M, size=max(n - len(pick), 0)).tolist())
+    return np.array(sorted(pick), dtype=np.int64)
+
+
+def run_gemm_case(oracle, M, N, K, bias: bool, seed: int, rows=None):
+    x = W.with_outliers((M, K), 0.01, 20.0, W._gen(seed, "cpu"), "cpu")
+    w = W.normal((N, K), 0.02, W._gen(seed + 1, "cpu"), "cpu").to(torch.bfloat16)
+    b = W.normal((N,), 0.01, W._gen(seed + 2, "cpu"), "cpu").to(torch.bfloat16) if bias else None
+    xp, xsf, gx = oracle.quantize(W.to_u16(x))
+    wp, wsf, gw = oracle.quantize(W.to_u16(w))
+    al = oracle.alpha(gx, gw)
+    y = nv.nvfp4_gemm(t(xp), t(xsf), t(wp), t(wsf), torch.tensor([al], device=DEV),
+                      None if b is None else b.to(DEV), M, N, K)
+    torch.cuda.synchronize()
+    assert nv.last_device_status() == nv.OK
+    y64 = oracle.gemm_f64(xp, xsf, wp, wsf, M, N, K, al, None if b is None else W.to_u16(b),
+                          rows=rows)
+    yg = y if rows is None else y[torch.from_numpy(rows).to(DEV)]
+    return assert_gemm_close(yg, y64, f"gemm M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (128, 256, 256),          # the tiny linear
+    (1, 8, 64), (2, 16, 64), (100, 200, 192), (129, 300, 320), (257, 513, 1024),
+    (300, 640, 576), (64, 128, 128), (256, 1000, 512), (384, 256, 2048),
+])
+@pytest.mark.parametrize("bias", [True, False])
+def test_gemm_parity(oracle, M, N, K, bias):
+    run_gemm_case(oracle, M, N, K, bias, seed=M * 31 + N * 7 + K)
+
+
+def test_gemm_vit_qkv_full_size(oracle):
+    """ViT block qkv projection: [32768, 1024] x [3072, 1024]^T, sampled rows."""
+    run_gemm_case(oracle, 32768, 3072, 1024, True, seed=11, rows=sample_rows(32768, 96))
+
+
+def test_gemm_down_proj_full_size(oracle):
+    """Qwen3-VL down_proj shape with the full K = 25600: [4096, 25600] x [5120, 25600]^T."""
+    run_gemm_case(oracle, 4096, 5120, 25600, False, seed=13, rows=sample_rows(4096, 12))
+
+
+def test_gemm_zero_sizes():
+    z = torch.zeros(16, dtype=torch.uint8, device=DEV)
+    a = torch.tensor([1.0], device=DEV)
+    y = torch.empty(16, dtype=torch.bfloat16, device=DEV)
+    L = nv.lib()
+    assert L.nvfp4_gemm(nv._ptr(z), nv._ptr(z), nv._ptr(z), nv._ptr(z), nv._ptr(a), None,
+                        nv._ptr(y), 0, 8, 64, nv._stream()) == nv.OK
+    assert L.nvfp4_gemm(nv._ptr(z), nv._ptr(z), nv._ptr(z), nv._ptr(z), nv._ptr(a), None,
+                        nv._ptr(y), 8, 0, 64, nv._stream()) == nv.OK
+
+
+@pytest.mark.parametrize("group", [0, 16, 128])
+@pytest.mark.parametrize("dynamic", [True, False])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (200, 384, 512), (33, 96, 1024)])
+def test_linear_parity(oracle, group, dynamic, M, N, K):
+    x = W.with_outliers((M, K), 0.01, 20.0, W._gen(M + N + K, "cpu"), "cpu")
+    w = W.normal((N, K), 0.02, W._gen(M + N + K + 1, "cpu"), "cpu").to(torch.bfloat16)
+    b = W.normal((N,), 0.01, W._gen(M + N + K + 2, "cpu"), "cpu").to(torch.bfloat16)
+    # weight: rotated (fold) and packed offline on the GPU, checked bit-exact first
+    wr_u16 = oracle.hadamard_rotate(W.to_u16(w), group) if group else W.to_u16(w)
+    wp, wsf, gw = nv.pack_weight(w.to(DEV), group)
+    owp, owsf, ogw = oracle.quantize(wr_u16)
+    assert np.array_equal(to_np(wp), owp) and np.array_equal(to_np(wsf), owsf)
+    gsf_x = None
+    if not dynamic:
+        xr = oracle.hadamard_rotate(W.to_u16(x), group) if group else W.to_u16(x)
+        gsf_x = oracle.global_scale(0.5 * oracle.amax_bf16(xr))      # calibrated too low: saturates
+    y = nv.nvfp4_linear(x.to(DEV), wp, wsf, gw, N, bias=b.to(DEV),
+                        gsf_x=None if gsf_x is None else torch.tensor([gsf_x], device=DEV),
+                        rotate_group=group)
+    torch.cuda.synchronize()
+    y64, *_ = oracle.linear(W.to_u16(x), owp, owsf, ogw, N, W.to_u16(b), gsf_x=gsf_x,
+                            rotate_group=group)
+    assert_gemm_close(y, y64, f"linear g={group} dynamic={dynamic}")
+
+
+def test_linear_vit_block_full_size(oracle):
+    """The four ViT-block linears at the 8-tile batch, g = 128, dynamic scale; sampled rows."""
+    for lin in W.vit_block("cpu"):
+        wp, wsf, gw = nv.pack_weight(lin.weight.to(DEV), 128)
+        y = nv.nvfp4_linear(lin.x.to(DEV), wp, wsf, gw, lin.N, bias=lin.bias.to(DEV),
+                            rotate_group=128)
+        torch.cuda.synchronize()
+        rows = sample_rows(lin.x.shape[0], 24, seed=lin.N)
+        y64, *_ = oracle.linear(W.to_u16(lin.x), to_np(wp), to_np(wsf), float(gw.item()), lin.N,
+                                W.to_u16(lin.bias), rotate_group=128, rows=rows)
+        assert_gemm_close(y[torch.from_numpy(rows).to(DEV)], y64, lin.name)
+
+
+def test_probe_error_on_gpu():
+    """The pages' probe through the GPU path: about 0.13 against the bf16 product."""
+    g = W._gen(1002, "cpu")
+    w = W.normal((1024, 5120), 0.02, g, "cpu").to(torch.bfloat16).to(DEV)
+    x = torch.randn(512, 5120, generator=W._gen(0, "cpu")).to(torch.bfloat16).to(DEV)
+    wp, wsf, gw = nv.pack_weight(w)
+    y = nv.nvfp4_linear(x, wp, wsf, gw, 1024, gsf_x=1.0)
+    ref = (x.double() @ w.double().T)
+    err = float((y.double() - ref).norm() / ref.norm())
+    assert abs(err - 0.13) < 0.02, err

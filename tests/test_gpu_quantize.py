@@ -1,0 +1,133 @@
+"""GPU parity of the quantizer, the amax pass and the Hadamard rotation against
+the CPU oracle, through the C ABI.  The bar is bit-exact: packed bytes, every
+scale byte including the padding, and the global-scale bit pattern.
+
+Pages: "minimax_h3_nvfp4_decoder" -- nvfp4_linear_inference (dynamic scale, 128x4
+layout), rotate_activation / from_linear (block Hadamard);
+"convert_minimax_h3_text_encoder_nvfp4.py" -- quantize_language_linear.
+"""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_17_b200 as nv
+from nvfp4_block_scaled_17_b200 import workloads as W
+from gpu_util import to_np
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def gpu_quantize(x: torch.Tensor, group: int, gsf):
+    R, K = x.shape
+    packed = torch.full((R, K // 2), 0xAB, dtype=torch.uint8, device=DEV)     # garbage first
+    sf = torch.full((nv.nvfp4_scale_bytes(R, K),), 0xAB, dtype=torch.uint8, device=DEV)
+    gsf_out = torch.full((1,), -7.0, dtype=torch.float32, device=DEV)
+    g_in = None if gsf is None else torch.tensor([gsf], dtype=torch.float32, device=DEV)
+    nv.nvfp4_quantize(x, group, g_in, out=(packed, sf, gsf_out))
+    torch.cuda.synchronize()
+    return to_np(packed), to_np(sf), np.float32(gsf_out.item())
+
+
+def oracle_quantize(oracle, x: torch.Tensor, group: int, gsf):
+    xu = W.to_u16(x)
+    if group:
+        xu = oracle.hadamard_rotate(xu, group)
+    return oracle.quantize(xu, gsf)
+
+
+def check(oracle, x, group, gsf):
+    p, s, g = gpu_quantize(x.to(DEV), group, gsf)
+    op, os_, og = oracle_quantize(oracle, x, group, gsf)
+    assert np.float32(og).view(np.uint32) == g.view(np.uint32), (og, g)
+    assert np.array_equal(s, os_), f"scale bytes differ at {np.flatnonzero(s != os_)[:8]}"
+    bad = np.argwhere(p != op)
+    assert bad.size == 0, f"{len(bad)} packed bytes differ, first {bad[:4].tolist()}"
+
+
+SHAPES = [(1, 16), (7, 48), (128, 256), (129, 80), (300, 1024), (33, 1040), (256, 128), (5, 2048)]
+
+
+@pytest.mark.parametrize("R,K", SHAPES)
+@pytest.mark.parametrize("dynamic", [True, False])
+def test_quantize_no_rotation(oracle, R, K, dynamic):
+    x = W.with_outliers((R, K), 0.01, 20.0, W._gen(R * 7 + K, "cpu"), "cpu")
+    gsf = None if dynamic else 2688.0 / 9.0
+    check(oracle, x, 0, gsf)
+
+
+@pytest.mark.parametrize("group", [16, 32, 64, 128])
+@pytest.mark.parametrize("R,K", [(1, 128), (130, 256), (64, 1024), (3, 384)])
+@pytest.mark.parametrize("dynamic", [True, False])
+def test_quantize_rotated(oracle, group, R, K, dynamic):
+    if K % group:
+        pytest.skip("K % group")
+    x = W.with_outliers((R, K), 0.005, 30.0, W._gen(R + K + group, "cpu"), "cpu")
+    check(oracle, x, group, None if dynamic else 37.5)
+
+
+def test_quantize_special_values(oracle):
+    R, K = 130, 192
+    x = torch.randn(R, K, generator=torch.Generator().manual_seed(5))
+    x[0] = 0                                # all-zero row
+    x[1, :16] = 0                           # all-zero block
+    x[2] *= 1e-30                           # tiny values (scale underflow)
+    x[3] *= 1e30                            # huge values
+    x[4, 5] = -0.0
+    x[5, :] = -1e-3                         # negative values rounding to zero codes
+    xb = x.to(torch.bfloat16)
+    check(oracle, xb, 0, None)
+    check(oracle, xb, 0, 1.0)               # unit scale (the pages' probe)
+    check(oracle, xb, 0, 1e6)               # static scale far too large: saturation
+    check(oracle, torch.zeros(3, 64, dtype=torch.bfloat16), 0, None)
+
+
+def test_quantize_vit_block_full_size(oracle):
+    """The 8-tile ViT-decoder activation [32768, 1024], g = 128, dynamic and static."""
+    lin = W.vit_block("cpu")[0]
+    check(oracle, lin.x, 128, None)
+    amax = float(oracle.amax_bf16(oracle.hadamard_rotate(W.to_u16(lin.x), 128)))
+    check(oracle, lin.x, 128, oracle.global_scale(amax))
+    check(oracle, lin.x, 0, None)
+
+
+def test_weight_pack_qwen_shape(oracle):
+    """Offline weight packing of one Qwen3-VL projection shape ([1024, 5120])."""
+    w = W.qwen3_weight((1024, 5120), "cpu", W._gen(3, "cpu"))
+    check(oracle, w, 0, None)
+
+
+@pytest.mark.parametrize("group", [16, 32, 64, 128])
+@pytest.mark.parametrize("R,K", [(1, 128), (129, 256), (64, 2048)])
+def test_hadamard_rotate(oracle, group, R, K):
+    x = W.random_bf16((R, K), seed=R * K + group)
+    y = nv.hadamard_rotate(x.to(DEV), group)
+    want = oracle.hadamard_rotate(W.to_u16(x), group)
+    assert np.array_equal(W.to_u16(y), want)
+    # in place
+    xi = x.to(DEV).clone()
+    nv.hadamard_rotate(xi, group, out=xi)
+    assert np.array_equal(W.to_u16(xi), want)
+
+
+def test_format_conversions_exhaustive(oracle):
+    """The quantizer's device fp32 -> E2M1 and fp32 -> E4M3 conversions against the
+    oracle's encoders on all 2^32 fp32 bit patterns (NaNs excluded)."""
+    n = 1 << 26
+    e2 = torch.empty(n, dtype=torch.uint8, device=DEV)
+    e4 = torch.empty(n, dtype=torch.uint8, device=DEV)
+    L = nv.lib()
+    for chunk in range(1 << 6):
+        first = chunk * n
+        assert L.nvfp4_debug_cvt_sweep(first, n, nv._ptr(e2), nv._ptr(e4), nv._stream()) == nv.OK
+        v = (np.arange(n, dtype=np.uint32) + np.uint32(first)).view(np.float32)
+        keep = ~np.isnan(v)
+        vk = v[keep]
+        g2, g4 = to_np(e2)[keep], to_np(e4)[keep]
+        o2 = oracle.e2m1_encode_array(vk)
+        bad2 = np.flatnonzero(g2 != o2)
+        assert bad2.size == 0, f"E2M1 differs for {vk[bad2[:6]]}: {g2[bad2[:6]]} vs {o2[bad2[:6]]}"
+        if first < (1 << 31):                 # E4M3 of |v|: the positive half covers it
+            o4 = oracle.e4m3_encode_array(vk)
+            bad4 = np.flatnonzero(g4 != o4)
+            assert bad4.size == 0, f"E4M3 differs for {vk[bad4[:6]]}: {g4[bad4[:6]]} vs {o4[bad4[:6]]}"
