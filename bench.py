@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 W4A4 linear on B200.
+
+Workload (one step): the four linears of one H3 ViT decoder block with 8 spatial
+tiles of 4096 tokens batched -- qkv [3072,1024], attn-out [1024,1024], FFN-in
+[4096,1024], FFN-out [1024,4096], M = 32768 -- each with a 128-wide block Hadamard
+folded into the weight, the dynamic activation scale (per-call amax), bias, bf16
+output.  Per linear the step runs the whole path: rotate + amax pass, rotate +
+quantize pass (nvfp4_quantize) and the block-scaled GEMM (nvfp4_gemm), exactly the
+launches nvfp4_linear makes, with CUDA events between them so the quantizer and the
+GEMM are timed separately on the launching stream.  Inputs are seeded synthetic
+tensors already in HBM; the activations of one step (448 MiB) exceed the 126 MB L2.
+
+Also measured in the same run: the static-scale variant of the step, offline weight
+packing (hadamard_rotate + nvfp4_quantize on the four weights), and the end-to-end
+path through nvfp4_linear with pinned host buffers (H2D of x and D2H of y inside the
+timed region).  The CPU baseline is the oracle on a bounded row sample.
+
+Prints one JSON line (rank 0).  --impl reference times the oracle instead.
+Multi-GPU (torchrun): every rank runs its own independent batch (weak scaling, no
+collective on the data path); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import nvfp4_block_scaled_17_b200 as nv  # noqa: E402
+from nvfp4_block_scaled_17_b200 import workloads as W  # noqa: E402
+
+METRIC = "nvfp4_linear TFLOPS (% of dense FP4 peak); quantizer GB/s (% of HBM)"
+GROUP = 128
+TOKENS = 8 * 4096
+CPU_SAMPLE_ROWS = 768
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return {"hbm": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
+                "bf16_sus": float(p["bf16_tflops_sustained"]), "src": "measured"}
+    except Exception:
+        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sus": 1400.0, "src": "fallback"}
+
+
+def workload_config(act_scale: str):
+    return {
+        "workload": "vit_decoder_block_8tiles",
+        "tokens": TOKENS,
+        "linears": [f"{n}[{N}x{K}]" for n, N, K in W.VIT_SHAPES],
+        "rotate_group": GROUP,
+        "act_scale": act_scale,
+        "bias": True,
+        "l2": "inputs larger than L2 (448 MiB of activations per step, 126 MB L2)",
+    }
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        rows = [ln.split(",") for ln in open(self.file.name).read().strip().splitlines() if ln.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our path
+# ---------------------------------------------------------------------------
+
+class Layer:
+    def __init__(self, lin: W.Linear, dev):
+        self.lin = lin
+        self.N, self.K = lin.N, lin.K
+        self.M = lin.x.shape[0]
+        self.x = lin.x
+        self.bias = lin.bias
+        self.wp, self.wsf, self.gsf_w = nv.pack_weight(lin.weight, GROUP)
+        self.xp = torch.empty(self.M, self.K // 2, dtype=torch.uint8, device=dev)
+        self.xsf = torch.empty(nv.nvfp4_scale_bytes(self.M, self.K), dtype=torch.uint8, device=dev)
+        self.scalars = torch.empty(2, dtype=torch.float32, device=dev)
+        self.ws = torch.empty(nv.nvfp4_quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+        self.y = torch.empty(self.M, self.N, dtype=torch.bfloat16, device=dev)
+        self.lin_ws = torch.empty(nv.nvfp4_linear_workspace_bytes(self.M, self.K),
+                                  dtype=torch.uint8, device=dev)
+        self.gsf_static = None
+
+    def flops(self):
+        return 2.0 * self.M * self.N * self.K
+
+    def quant_bytes(self, dynamic: bool, l2_bytes: int):
+        n = self.M * self.K
+        reads = 2.0 if (dynamic and 2 * n > l2_bytes // 2) else 1.0
+        return n * (2.0 * reads + 0.5) + nv.nvfp4_scale_bytes(self.M, self.K)
+
+
+def run_step(layers, dynamic: bool, events=None):
+    """One pass of the path over the four linears -- the same two entry points and three
+    launches per linear that nvfp4_linear makes (amax + quantize writing alpha, then the
+    GEMM); events[i] = (e0, e1, e2) per linear bracket the quantizer and the GEMM."""
+    L = nv.lib()
+    s = nv._stream()
+    for i, ly in enumerate(layers):
+        if events is not None:
+            events[i][0].record()
+        gsf_in = None if dynamic else ly.gsf_static
+        st = L.nvfp4_quantize(nv._ptr(ly.x), ly.M, ly.K, GROUP, nv._ptr(gsf_in),
+                              nv._ptr(ly.scalars[:1]), nv._ptr(ly.xp), nv._ptr(ly.xsf),
+                              nv._ptr(ly.gsf_w), nv._ptr(ly.scalars[1:]), nv._ptr(ly.ws),
+                              ly.ws.numel(), s)
+        if st:
+            raise nv.NVFP4Error("nvfp4_quantize", st)
+        if events is not None:
+            events[i][1].record()
+        st = L.nvfp4_gemm(nv._ptr(ly.xp), nv._ptr(ly.xsf), nv._ptr(ly.wp), nv._ptr(ly.wsf),
+                          nv._ptr(ly.scalars[1:]), nv._ptr(ly.bias), nv._ptr(ly.y), ly.M, ly.N,
+                          ly.K, s)
+        if st:
+            raise nv.NVFP4Error("nvfp4_gemm", st)
+        if events is not None:
+            events[i][2].record()
+
+
+def timed_steps(layers, dynamic, steps, warmup, dist_on):
+    for _ in range(warmup):
+        run_step(layers, dynamic)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in layers]
+           for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for k in range(steps):
+        run_step(layers, dynamic, evs[k])
+    stop.record()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(stop)
+    q_ms = [sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(steps)) / steps
+            for i in range(len(layers))]
+    g_ms = [sum(evs[k][i][1].elapsed_time(evs[k][i][2]) for k in range(steps)) / steps
+            for i in range(len(layers))]
+    return total_ms, q_ms, g_ms
+
+
+def max_over_ranks(v: float, dist_on: bool) -> float:
+    if not dist_on:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def e2e_steps(layers, steps, warmup, dist_on):
+    """Through the public nvfp4_linear call with pinned host buffers: per step, H2D of
+    every linear's x, the linear, D2H of every y (all on the current stream)."""
+    host_x = [ly.x.cpu().pin_memory() for ly in layers]
+    host_y = [torch.empty(ly.y.shape, dtype=torch.bfloat16).pin_memory() for ly in layers]
+    dev_x = [torch.empty_like(ly.x) for ly in layers]
+
+    def step():
+        for i, ly in enumerate(layers):
+            dev_x[i].copy_(host_x[i], non_blocking=True)
+            nv.nvfp4_linear(dev_x[i], ly.wp, ly.wsf, ly.gsf_w, ly.N, bias=ly.bias,
+                            rotate_group=GROUP, workspace=ly.lin_ws, out=ly.y)
+            host_y[i].copy_(ly.y, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    start.record()
+    for _ in range(steps):
+        step()
+    stop.record()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    ms = max_over_ranks(start.elapsed_time(stop) / steps, dist_on)
+    h2d = sum(x.numel() * 2 for x in host_x)
+    d2h = sum(y.numel() * 2 for y in host_y)
+    return ms, h2d, d2h
+
+
+def weight_pack_rate(layers_src, dev):
+    """Offline packing of the four weights (rotate + dynamic-scale quantize), GB/s over
+    the algorithmic bytes: rotate 4 B/value, amax 2 B/value, quantize 2.5625 B/value."""
+    ws = [l.weight for l in layers_src]
+    for w in ws:
+        nv.pack_weight(w, GROUP)
+    torch.cuda.synchronize()
+    reps = 10
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        for w in ws:
+            nv.pack_weight(w, GROUP)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    n = sum(w.numel() for w in ws)
+    byts = n * (4.0 + 2.0 + 2.5625)
+    return {"values": n, "ms": ms, "GBps": byts / (ms * 1e-3) / 1e9,
+            "bytes_per_value": 8.5625}
+
+
+def cpu_baseline(layers_src, rows: int):
+    """The oracle as it stands on the host cores: rotate, dynamic quantize and the fp64
+    GEMM for `rows` rows of each linear (weights packed by the oracle, untimed)."""
+    import numpy as np
+
+    import oracle as O
+    O.build()
+    packed = []
+    for l in layers_src:
+        wr = O.hadamard_rotate(W.to_u16(l.weight), GROUP)
+        packed.append(O.quantize(wr))
+    xs = [W.to_u16(l.x[:rows]) for l in layers_src]
+    bs = [W.to_u16(l.bias) for l in layers_src]
+    t0 = time.perf_counter()
+    flops = 0.0
+    for l, (wp, wsf, gw), x, b in zip(layers_src, packed, xs, bs):
+        O.linear(x, wp, wsf, gw, l.N, b, rotate_group=GROUP)
+        flops += 2.0 * rows * l.N * l.K
+    dt = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{rows} rows of each of the 4 linears (rotate g=128, dynamic quantize, "
+                      f"fp64 GEMM over all N), {dt:.1f} s"}, dt
+
+
+def run_ours(args, dist_on, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 1024 * 1024))
+    pk = peaks()
+    src = W.vit_block(dev, seed=1001 + rank, tokens=TOKENS)
+    layers = [Layer(l, dev) for l in src]
+    # static scale: the scale a calibration pass over this very input would store, i.e.
+    # the dynamic scale of one untimed call
+    for ly in layers:
+        _, _, g = nv.nvfp4_quantize(ly.x, GROUP, None)
+        ly.gsf_static = g
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    if not args.kernels_only:
+        clocks.start()
+    total_ms, q_ms, g_ms = timed_steps(layers, True, args.steps, args.warmup, dist_on)
+    clk = None if args.kernels_only else clocks.stop()
+    if args.kernels_only:        # profiling runs: the dynamic-scale step only
+        s_total, s_q, s_g = total_ms, q_ms, g_ms
+        e2e_ms, h2d, d2h, wpack = float("nan"), 0, 0, None
+    else:
+        s_total, s_q, s_g = timed_steps(layers, False, args.steps, args.warmup, dist_on)
+        e2e_ms, h2d, d2h = e2e_steps(layers, max(2, args.steps // 4), max(3, args.warmup),
+                                     dist_on)
+        wpack = weight_pack_rate(src, dev)
+    assert nv.last_device_status() == nv.OK
+
+    ms = max_over_ranks(total_ms / args.steps, dist_on)
+    s_ms = max_over_ranks(s_total / args.steps, dist_on)
+    flops = sum(ly.flops() for ly in layers)
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    fp4_peak = 4.0 * pk["bf16_sus"]           # nominal fp4 / bf16 = 9 / 2.25
+    g_time = sum(g_ms)
+    gemm_tflops = flops / (g_time * 1e-3) / 1e12
+    q_bytes = sum(ly.quant_bytes(True, l2) for ly in layers)
+    q_time = sum(q_ms)
+    q_gbps = q_bytes / (q_time * 1e-3) / 1e9
+    dominant_is_gemm = g_time >= q_time
+    gemm_roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                 "frac": gemm_tflops / fp4_peak, "traffic": None, "kernel": "gemm_kernel",
+                 "per_linear_ms": g_ms,
+                 "peak_note": f"{pk['src']}: 4 x bf16 sustained ({pk['bf16_sus']} TFLOP/s), "
+                              "nominal dense fp4/bf16 ratio 9/2.25; burst-based frac "
+                              f"{gemm_tflops / (4 * pk['bf16']):.3f}"}
+    quant_roof = {"bound": "hbm", "achieved": q_gbps, "peak": pk["hbm"], "unit": "GB/s",
+                  "frac": q_gbps / pk["hbm"], "traffic": None, "kernel": "unit_kernel (amax + quantize)",
+                  "per_linear_ms": q_ms,
+                  "bytes_note": "4.5625 B/value (two reads of x, dynamic scale, x > L2/2) + scales",
+                  "peak_note": f"{pk['src']} copy bandwidth; frac of 8 TB/s: {q_gbps / 8000:.3f}"}
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3/16, fp32 accumulate)",
+        "data": "synthetic (seeded; N(0,1) activations with 0.5% outliers x30, N(0,0.02) weights)",
+        "config": workload_config("dynamic"),
+        "roofline": gemm_roof if dominant_is_gemm else quant_roof,
+        "roofline_gemm": gemm_roof, "roofline_quantizer": quant_roof,
+        "static_scale": {"ms_per_step": s_ms, "TFLOP/s": world * flops / (s_ms * 1e-3) / 1e12,
+                         "quantizer_ms": s_q, "gemm_ms": s_g},
+        "weight_pack": wpack,
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "nvfp4_linear"},
+        "gpu_launches": 3 * len(layers) * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.kernels_only):
+        cb, _ = cpu_baseline(src, CPU_SAMPLE_ROWS)
+        out["cpu_baseline"] = cb
+    return out
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step is a bounded sample of the same
+    workload (rows of each linear) on the host cores; rank 0 only."""
+    if rank != 0:
+        return None
+    src = W.vit_block("cpu", seed=1001, tokens=CPU_SAMPLE_ROWS)
+    for _ in range(args.warmup):
+        cpu_baseline(src, 32)
+    vals, dts = [], []
+    for _ in range(args.steps):
+        cb, dt = cpu_baseline(src, CPU_SAMPLE_ROWS // 4)
+        vals.append(cb["value"])
+        dts.append(dt)
+    v = statistics.mean(vals)
+    cb["value"] = v
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(dts),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": workload_config("dynamic"),
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernels-only", action="store_true",
+                    help="time only the dynamic-scale step (for profiler runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    if dist_on:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    out = run_ours(args, dist_on, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

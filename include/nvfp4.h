@@ -114,6 +114,10 @@ NVFP4_API size_t nvfp4_quantize_workspace_bytes(void);
  *                  (may be NULL when gsf_in is given)
  *   packed       : out, uint8 [rows, K/2]
  *   sf           : out, uint8 [nvfp4_scale_bytes(rows, K)], padding written as 0
+ *   gsf_w        : in,  optional device fp32 scalar (the weight's global scale of the
+ *                  GEMM this activation feeds); with alpha_out, the kernel also writes
+ *   alpha_out    : out, optional device fp32 scalar alpha = rn(1 / rn(gsf * gsf_w)),
+ *                  ready for nvfp4_gemm; both NULL or both given
  *   workspace    : scratch of nvfp4_quantize_workspace_bytes() bytes (dynamic only;
  *                  may be NULL for a static call), 16-byte aligned, caller-owned,
  *                  contents need no initialisation
@@ -123,8 +127,9 @@ NVFP4_API size_t nvfp4_quantize_workspace_bytes(void);
  * Errors: INVALID_ARG, SHAPE (K <= 0, K % 16, K % group), ALIGN, WORKSPACE, DEVICE, CUDA.
  */
 NVFP4_API nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t K, int rotate_group,
-                            const float* gsf_in, float* gsf_out, uint8_t* packed, uint8_t* sf,
-                            void* workspace, size_t ws_bytes, void* stream);
+                                      const float* gsf_in, float* gsf_out, uint8_t* packed,
+                                      uint8_t* sf, const float* gsf_w, float* alpha_out,
+                                      void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * nvfp4_gemm -- block-scaled FP4 GEMM on the tcgen05 tensor cores with the

@@ -32,7 +32,8 @@ SIGNATURES = {
     "nvfp4_packed_bytes": (_sz, [_i64, _i64]),
     "hadamard_rotate": (_int, [_vp, _vp, _i64, _i64, _int, _vp]),
     "nvfp4_quantize_workspace_bytes": (_sz, []),
-    "nvfp4_quantize": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_quantize": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                              _vp]),
     "nvfp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64]),
     "nvfp4_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _int, _vp, _sz, _vp,
@@ -134,10 +135,13 @@ def hadamard_rotate(x: torch.Tensor, group: int, out: torch.Tensor | None = None
 
 
 def nvfp4_quantize(x: torch.Tensor, rotate_group: int = 0, gsf: torch.Tensor | float | None = None,
-                   out: tuple | None = None, workspace: torch.Tensor | None = None, stream=None):
+                   out: tuple | None = None, workspace: torch.Tensor | None = None,
+                   gsf_w: torch.Tensor | None = None, alpha_out: torch.Tensor | None = None,
+                   stream=None):
     """bf16 [rows, K] -> (packed uint8 [rows, K/2], scales uint8 [scale_bytes], gsf fp32 [1]).
 
-    gsf=None computes the dynamic global scale 2688/amax over the whole tensor."""
+    gsf=None computes the dynamic global scale 2688/amax over the whole tensor.  With
+    gsf_w and alpha_out the kernel also writes alpha = 1/(gsf * gsf_w) for nvfp4_gemm."""
     _bf16_2d(x, "x")
     R, K = x.shape
     gsf_in = _scalar(gsf, x.device, "gsf")
@@ -152,7 +156,7 @@ def nvfp4_quantize(x: torch.Tensor, rotate_group: int = 0, gsf: torch.Tensor | f
         ws = torch.empty(nvfp4_quantize_workspace_bytes(), dtype=torch.uint8, device=x.device)
     _check("nvfp4_quantize", lib().nvfp4_quantize(
         _ptr(x), R, K, int(rotate_group), _ptr(gsf_in), _ptr(gsf_out), _ptr(packed), _ptr(sf),
-        _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+        _ptr(gsf_w), _ptr(alpha_out), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return packed, sf, gsf_out
 
 

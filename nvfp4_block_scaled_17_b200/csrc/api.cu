@@ -127,9 +127,13 @@ size_t nvfp4_quantize_workspace_bytes(void) { return kQuantWorkspace; }
 
 nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int group,
                             const float* gsf_in, float* gsf_out, uint8_t* packed, uint8_t* sf,
-                            void* workspace, size_t ws_bytes, void* stream) {
+                            const float* gsf_w, float* alpha_out, void* workspace,
+                            size_t ws_bytes, void* stream) {
     if (!x || !packed || !sf || rows < 0 || !valid_group(group)) return NVFP4_ERR_INVALID_ARG;
     if (!gsf_in && !gsf_out) return NVFP4_ERR_INVALID_ARG;
+    if ((gsf_w == nullptr) != (alpha_out == nullptr)) return NVFP4_ERR_INVALID_ARG;
+    if ((gsf_w && !aligned(gsf_w, 4)) || (alpha_out && !aligned(alpha_out, 4)))
+        return NVFP4_ERR_ALIGN;
     if (K <= 0 || K % 16 || (group && K % group)) return NVFP4_ERR_SHAPE;
     if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(sf, 16)) return NVFP4_ERR_ALIGN;
     if ((gsf_in && !aligned(gsf_in, 4)) || (gsf_out && !aligned(gsf_out, 4)))
@@ -143,7 +147,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t K, int group,
     if (st != NVFP4_OK) return st;
     if (rows == 0) return NVFP4_OK;
     return launch_quantize(x, rows, K, group, gsf_in, gsf_out, packed, sf,
-                           static_cast<float*>(workspace), nullptr, nullptr,
+                           static_cast<float*>(workspace), gsf_w, alpha_out,
                            static_cast<cudaStream_t>(stream));
 }
 

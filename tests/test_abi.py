@@ -58,16 +58,17 @@ def test_sizes_match_oracle(L, oracle):
 
 def test_quantize_argument_errors(L):
     q = L.nvfp4_quantize
-    assert q(None, 4, 64, 0, A, A, A, A, A, 4096, S) == nv.ERR_INVALID_ARG
-    assert q(A, -1, 64, 0, A, A, A, A, A, 4096, S) == nv.ERR_INVALID_ARG
-    assert q(A, 4, 64, 8, A, A, A, A, A, 4096, S) == nv.ERR_INVALID_ARG      # group 8
-    assert q(A, 4, 64, 0, None, None, A, A, A, 4096, S) == nv.ERR_INVALID_ARG  # no scale at all
-    assert q(A, 4, 24, 0, A, A, A, A, A, 4096, S) == nv.ERR_SHAPE            # K % 16
-    assert q(A, 4, 0, 0, A, A, A, A, A, 4096, S) == nv.ERR_SHAPE
-    assert q(A, 4, 96, 64, A, A, A, A, A, 4096, S) == nv.ERR_SHAPE           # K % group
-    assert q(MIS, 4, 64, 0, A, A, A, A, A, 4096, S) == nv.ERR_ALIGN
-    assert q(A, 4, 64, 0, None, A, A, A, None, 0, S) == nv.ERR_WORKSPACE     # dynamic, no scratch
-    assert q(A, 4, 64, 0, None, A, A, A, A, 16, S) == nv.ERR_WORKSPACE
+    assert q(None, 4, 64, 0, A, A, A, A, None, None, A, 4096, S) == nv.ERR_INVALID_ARG
+    assert q(A, -1, 64, 0, A, A, A, A, None, None, A, 4096, S) == nv.ERR_INVALID_ARG
+    assert q(A, 4, 64, 8, A, A, A, A, None, None, A, 4096, S) == nv.ERR_INVALID_ARG      # group 8
+    assert q(A, 4, 64, 0, None, None, A, A, None, None, A, 4096, S) == nv.ERR_INVALID_ARG  # no scale at all
+    assert q(A, 4, 24, 0, A, A, A, A, None, None, A, 4096, S) == nv.ERR_SHAPE            # K % 16
+    assert q(A, 4, 0, 0, A, A, A, A, None, None, A, 4096, S) == nv.ERR_SHAPE
+    assert q(A, 4, 96, 64, A, A, A, A, None, None, A, 4096, S) == nv.ERR_SHAPE           # K % group
+    assert q(MIS, 4, 64, 0, A, A, A, A, None, None, A, 4096, S) == nv.ERR_ALIGN
+    assert q(A, 4, 64, 0, None, A, A, A, None, None, None, 0, S) == nv.ERR_WORKSPACE     # dynamic, no scratch
+    assert q(A, 4, 64, 0, None, A, A, A, None, None, A, 16, S) == nv.ERR_WORKSPACE
+    assert q(A, 4, 64, 0, A, A, A, A, A, None, None, 0, S) == nv.ERR_INVALID_ARG  # gsf_w alone
 
 
 def test_gemm_and_linear_argument_errors(L):
