@@ -40,6 +40,28 @@ import nvfp4_block_scaled_17_b200 as nv  # noqa: E402
 from nvfp4_block_scaled_17_b200 import workloads as W  # noqa: E402
 
 METRIC = "nvfp4_linear TFLOPS (% of dense FP4 peak); quantizer GB/s (% of HBM)"
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one step, from the ncu
+# captures summarised in profiles/ (gemm_kernel_vit_block.md, unit_kernel_vit_qkv.md),
+# valid only for the kernel sources they were taken on (sha256 prefix); reported as
+# null once the source has changed.  The quantizer figure is the qkv launch pair scaled
+# by the step's value count (traffic grows in proportion to the values).
+MEASURED_TRAFFIC = {
+    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "88cf5ad9245bf369",
+             "bytes_per_step": 545.6e6},
+    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "0099cc90a1a01db0",
+              "bytes_per_step": 138.1e6 * (3 * 32768 * 1024 + 32768 * 4096) / (32768 * 1024)},
+}
+
+
+def measured_traffic(key):
+    import hashlib
+    t = MEASURED_TRAFFIC[key]
+    try:
+        sha = hashlib.sha256(open(os.path.join(ROOT, t["src"]), "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return t["bytes_per_step"] if sha == t["sha"] else None
 GROUP = 128
 TOKENS = 8 * 4096
 CPU_SAMPLE_ROWS = 768
@@ -332,13 +354,16 @@ def run_ours(args, dist_on, rank, world, local_rank):
     q_gbps = q_bytes / (q_time * 1e-3) / 1e9
     dominant_is_gemm = g_time >= q_time
     gemm_roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                 "frac": gemm_tflops / fp4_peak, "traffic": None, "kernel": "gemm_kernel",
-                 "per_linear_ms": g_ms,
+                 "frac": gemm_tflops / fp4_peak, "traffic": measured_traffic("gemm"),
+                 "traffic_unit": "bytes per step (4 launches)", "kernel": "gemm_kernel",
+                 "per_linear_ms": g_ms, "algorithmic_flop": flops,
                  "peak_note": f"{pk['src']}: 4 x bf16 sustained ({pk['bf16_sus']} TFLOP/s), "
                               "nominal dense fp4/bf16 ratio 9/2.25; burst-based frac "
                               f"{gemm_tflops / (4 * pk['bf16']):.3f}"}
     quant_roof = {"bound": "hbm", "achieved": q_gbps, "peak": pk["hbm"], "unit": "GB/s",
-                  "frac": q_gbps / pk["hbm"], "traffic": None, "kernel": "unit_kernel (amax + quantize)",
+                  "frac": q_gbps / pk["hbm"], "traffic": measured_traffic("quant"),
+                  "traffic_unit": "bytes per step (8 launches)", "algorithmic_bytes": q_bytes,
+                  "kernel": "unit_kernel (amax + quantize)",
                   "per_linear_ms": q_ms,
                   "bytes_note": "4.5625 B/value (two reads of x, dynamic scale, x > L2/2) + scales",
                   "peak_note": f"{pk['src']} copy bandwidth; frac of 8 TB/s: {q_gbps / 8000:.3f}"}

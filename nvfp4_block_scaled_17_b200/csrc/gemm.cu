@@ -11,13 +11,23 @@
 //               256 x 128-byte B box (128-byte swizzle), plus the matching 512-byte
 //               chunks of the 128x4 scale layout with plain bulk copies (the layout
 //               already is the tensor-memory copy order, so no reshuffle is needed).
-//   warp 1      MMA issuer (one lane): tcgen05.cp of the scale chunks into tensor
-//               memory, then tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64)
-//               four times per stage, accumulating in tensor memory; tcgen05.commit
-//               releases the stage and, at the end of a tile, hands the accumulator to
-//               the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quadrant, alpha, bias, bf16,
-//               stores.
+//   warp 1      MMA issuer (one lane): per K=64 step, tcgen05.cp of the step's scale
+//               chunks into a ring of five tensor-memory slots, then tcgen05.mma
+//               kind::mxf4nvf4 block16 (M=128, N=256, K=64), accumulating in tensor
+//               memory; tcgen05.commit releases the stage and, at the end of a tile,
+//               hands the accumulator to the epilogue.  The copy for step g overwrites
+//               the slot of step g-5, long finished, so the in-order tensor pipe never
+//               waits for an MMA to stop reading the scales it is about to replace.
+//   warps 2..9  epilogue, two warps per 32-lane tensor-memory quadrant (one per
+//               128-column half): tcgen05.ld, alpha, bias, bf16, a 64-byte-swizzled
+//               shared staging tile, TMA store (bounds clipped by the tensor map).
+//
+// Accumulator double buffering within 512 tensor-memory columns: tile buffers
+// occupy columns [0, 256) and [192, 448), the scale-factor ring [448, 508).  The two
+// buffers share columns [192, 256); the epilogue drains that shared part of a tile
+// first and releases it, so the MMAs of the next tile start while the rest of the
+// previous accumulator is still being stored.
+//
 // Every wait is bounded (globaltimer); on expiry the kernel records
 // NVFP4_ERR_TIMEOUT, drains its own copies and MMAs, frees tensor memory and exits.
 // No load uses cluster multicast.
@@ -33,16 +43,21 @@ namespace {
 constexpr int BM = 128;                 // rows of A per tile (= tensor-memory lanes)
 constexpr int BN = 256;                 // rows of B per tile (= accumulator columns)
 constexpr int BKB = 128;                // bytes of packed K per stage (256 values)
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int SMEM_A = BM * BKB;        // 16 KiB
 constexpr int SMEM_B = BN * BKB;        // 32 KiB
 constexpr int SMEM_SFA = 4 * 512;       // four K=64 scale chunks for 128 rows
 constexpr int SMEM_SFB = 8 * 512;       // the same for 256 rows (two 128-row tiles)
+constexpr int STG_BYTES = 32 * 64;      // one 32 x 32 bf16 staging tile
+constexpr int SMEM_STG = EPI_WARPS * 2 * STG_BYTES;
+constexpr int SMEM_BYTES =
+    1024 + STAGES * (SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB) + SMEM_STG + 256;
 constexpr int TMEM_COLS = 512;
-constexpr int TMEM_SFA = 256;           // 4 chunks x 4 columns
-constexpr int TMEM_SFB = 272;           // 4 chunks x 8 columns
-constexpr int THREADS = 192;
-constexpr int SMEM_BYTES = 1024 + STAGES * (SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB) + 256;
+constexpr uint32_t TMEM_BUF1 = 192;     // second accumulator buffer (overlaps [192, 256))
+constexpr uint32_t TMEM_SF = 448;       // ring of scale-factor slots
+constexpr int SF_SLOTS = 5;             // 12 columns each: 4 for A, 8 for B (256 rows)
 
 // Instruction descriptor: E2M1 x E2M1 (format 1), both K-major, UE4M3 scales,
 // N = 256, M = 128, dense K = 64.
@@ -60,29 +75,44 @@ struct GemmParams {
     int k_tiles;               // ceil(K / 256)
     int kchunks;               // K / 64: scale chunks per 128-row tile
     int sf_row_tiles_b;        // ceil(N / 128)
+    int tma_store;             // 1: y through the tensor map (N % 8 == 0)
+    int n_fast;                // tile order: 1 = consecutive tiles walk N (B re-read from L2)
     int* status;
     uint64_t budget_ns;
 };
 
-__device__ __forceinline__ uint16_t bf16_bits_rn(float v) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) { return bf16x2_rn(lo, hi); }
+
+// Tile order.  The CTAs of one wave work on consecutive tiles; walking N first keeps
+// the few A row blocks of a wave hot while the (smaller) B panel is re-read from L2,
+// walking M first does the opposite.
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& m_blk, int& n_blk) {
+    if (p.n_fast) {
+        n_blk = tile % p.n_blocks;
+        m_blk = tile / p.n_blocks;
+    } else {
+        m_blk = tile % p.m_blocks;
+        n_blk = tile / p.m_blocks;
+    }
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            const GemmParams p) {
+            const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + STAGES * SMEM_A;
-    uint8_t* sSFA = sB + STAGES * SMEM_B;
+    uint8_t* sStg = sB + STAGES * SMEM_B;
+    uint8_t* sSFA = sStg + SMEM_STG;
     uint8_t* sSFB = sSFA + STAGES * SMEM_SFA;
     uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SMEM_SFB);
     uint64_t* empty = full + STAGES;
-    uint64_t* acc_full = empty + STAGES;
-    uint64_t* acc_empty = acc_full + 1;
-    uint64_t* drain = acc_empty + 1;
+    uint64_t* acc_full = empty + STAGES;     // [2]
+    uint64_t* acc_free = acc_full + 2;       // [2]
+    uint64_t* ovl_free = acc_free + 2;
+    uint64_t* drain = ovl_free + 1;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -94,8 +124,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_free[b], EPI_WARPS);
+        }
+        mbar_init(ovl_free, EPI_WARPS / 2);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -117,8 +150,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             uint32_t issued = 0, issued_phase = 0;   // per-stage bit masks
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                const int m_blk = tile % p.m_blocks;
-                const int n_blk = tile / p.m_blocks;
+                int m_blk, n_blk;
+                tile_coords(p, tile, m_blk, n_blk);
                 const int sfb_tiles = (2 * n_blk + 1 < p.sf_row_tiles_b) ? 2 : 1;
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status,
@@ -157,17 +190,23 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     } else if (warp == 1) {
         if (lane == 0) {
             int stage = 0;
-            uint32_t phase = 0, acc_phase = 0;
+            uint32_t phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                const int n_blk = tile / p.m_blocks;
-                (void)n_blk;
-                if (!mbar_wait_bounded(acc_empty, acc_phase ^ 1, abort_flag, p.status,
+            int it = 0;
+            int sf_slot = 0;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+                const int b = it & 1;
+                const uint32_t use = (uint32_t)(it >> 1);
+                // buffer b fully drained (tile it-2) and the shared columns drained (tile it-1)
+                if (!mbar_wait_bounded(&acc_free[b], (use & 1) ^ 1, abort_flag, p.status,
+                                       p.budget_ns) ||
+                    !mbar_wait_bounded(ovl_free, (uint32_t)(it & 1) ^ 1, abort_flag, p.status,
                                        p.budget_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t acc = tmem + (b ? TMEM_BUF1 : 0u);
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status,
                                            p.budget_ns)) {
@@ -181,14 +220,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     const uint32_t sfa0 = smem_u32(sSFA + stage * SMEM_SFA);
                     const uint32_t sfb0 = smem_u32(sSFB + stage * SMEM_SFB);
                     for (int kk = 0; kk < steps; ++kk) {
-                        tc_copy_sf(tmem + TMEM_SFA + 4 * kk, sdesc_sf(sfa0 + 512 * kk));
-                        tc_copy_sf(tmem + TMEM_SFB + 8 * kk, sdesc_sf(sfb0 + 512 * kk));
-                        tc_copy_sf(tmem + TMEM_SFB + 8 * kk + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
-                    }
-                    for (int kk = 0; kk < steps; ++kk) {
-                        mma_nvf4(tmem, sdesc_kmajor_sw128(a0 + 32 * kk),
-                                 sdesc_kmajor_sw128(b0 + 32 * kk), IDESC, tmem + TMEM_SFA + 4 * kk,
-                                 tmem + TMEM_SFB + 8 * kk, (kt | kk) != 0);
+                        const uint32_t sfa_t = tmem + TMEM_SF + 12u * (uint32_t)sf_slot;
+                        const uint32_t sfb_t = sfa_t + 4;
+                        tc_copy_sf(sfa_t, sdesc_sf(sfa0 + 512 * kk));
+                        tc_copy_sf(sfb_t, sdesc_sf(sfb0 + 512 * kk));
+                        tc_copy_sf(sfb_t + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
+                        mma_nvf4(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
+                                 sdesc_kmajor_sw128(b0 + 32 * kk), IDESC, sfa_t, sfb_t,
+                                 (kt | kk) != 0);
+                        if (++sf_slot == SF_SLOTS) sf_slot = 0;
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == STAGES) {
@@ -197,8 +237,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     }
                 }
                 if (!ok) break;
-                tc_commit(acc_full);
-                acc_phase ^= 1;
+                tc_commit(&acc_full[b]);
             }
             // Wait until every tensor-core operation this thread issued has finished.
             tc_commit(drain);
@@ -207,55 +246,104 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         }
         __syncwarp();
     } else {
-        // epilogue: warp w reads tensor-memory lanes 32*(w%4) .. 32*(w%4)+31
+        // epilogue: quadrant q = warp % 4 (tensor-memory lanes 32q..32q+31), column half h
         const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;
         const float alpha = *p.alpha;
-        const bool vec_ok = (p.N % 8) == 0;
-        uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            const int m_blk = tile % p.m_blocks;
-            const int n_blk = tile / p.m_blocks;
-            if (!mbar_wait_bounded(acc_full, acc_phase, abort_flag, p.status, p.budget_ns)) break;
+        uint8_t* stg = sStg + (warp - 2) * 2 * STG_BYTES;
+        int stg_sel = 0;
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+            int m_blk, n_blk;
+            tile_coords(p, tile, m_blk, n_blk);
+            const int b = it & 1;
+            const uint32_t use = (uint32_t)(it >> 1);
+            if (!mbar_wait_bounded(&acc_full[b], use & 1, abort_flag, p.status, p.budget_ns)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
-            const int row = m_blk * BM + quad * 32 + lane;
-            uint16_t* yrow = p.y + (size_t)row * p.N;
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                const int n0 = n_blk * BN + c0;
-                if (n0 >= p.N) break;   // warp-uniform
-                uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, r);
-                tmem_ld_wait();
-                uint32_t packed[16];
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    float v0 = __fmul_rn(alpha, __uint_as_float(r[j]));
-                    float v1 = __fmul_rn(alpha, __uint_as_float(r[j + 1]));
+            // The shared columns [192, 256) are chunks 6, 7 of buffer 0 (half 1) and chunks
+            // 0, 1 of buffer 1 (half 0): the owning half drains them first.
+            const bool owns_overlap = (b == 0) ? (half == 1) : (half == 0);
+            const uint32_t buf_col = b ? TMEM_BUF1 : 0u;
+            const int row0 = m_blk * BM + quad * 32;
+            for (int i = 0; i < 4; ++i) {
+                const int chunk = (b == 0 && half == 1) ? ((i + 2) & 3) + 4 : half * 4 + i;
+                const int n0 = n_blk * BN + chunk * 32;
+                if (n0 < p.N) {   // warp-uniform
+                    uint32_t r[32];
+                    tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + buf_col + (uint32_t)chunk * 32, r);
+                    tmem_ld_wait();
+                    float bv[32];
                     if (p.bias) {
-                        const int na = min(n0 + j, p.N - 1), nb = min(n0 + j + 1, p.N - 1);
-                        v0 = __fadd_rn(v0, __uint_as_float((uint32_t)p.bias[na] << 16));
-                        v1 = __fadd_rn(v1, __uint_as_float((uint32_t)p.bias[nb] << 16));
-                    }
-                    packed[j / 2] = (uint32_t)bf16_bits_rn(v0) | ((uint32_t)bf16_bits_rn(v1) << 16);
-                }
-                if (row < p.M) {
-                    if (vec_ok && n0 + 32 <= p.N) {
-                        uint4* d = reinterpret_cast<uint4*>(yrow + n0);
+                        if (n0 + 32 <= p.N) {
+                            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            d[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
-                                              packed[4 * q + 3]);
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                const uint4 w = bp[q4];
+                                bv[8 * q4 + 0] = bf16lo(w.x); bv[8 * q4 + 1] = bf16hi(w.x);
+                                bv[8 * q4 + 2] = bf16lo(w.y); bv[8 * q4 + 3] = bf16hi(w.y);
+                                bv[8 * q4 + 4] = bf16lo(w.z); bv[8 * q4 + 5] = bf16hi(w.z);
+                                bv[8 * q4 + 6] = bf16lo(w.w); bv[8 * q4 + 7] = bf16hi(w.w);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                bv[j] = __uint_as_float((uint32_t)p.bias[min(n0 + j, p.N - 1)] << 16);
+                        }
+                    }
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        float v0 = __fmul_rn(alpha, __uint_as_float(r[j]));
+                        float v1 = __fmul_rn(alpha, __uint_as_float(r[j + 1]));
+                        if (p.bias) {
+                            v0 = __fadd_rn(v0, bv[j]);
+                            v1 = __fadd_rn(v1, bv[j + 1]);
+                        }
+                        packed[j / 2] = bf16x2_bits(v0, v1);
+                    }
+                    if (p.tma_store) {
+                        uint8_t* sb = stg + stg_sel * STG_BYTES;
+                        if (lane == 0) bulk_wait_read<1>();   // this buffer's previous store
+                        __syncwarp();
+                        // 64-byte swizzle: 16-byte chunk c of row r sits at c ^ ((r >> 1) & 3)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4*>(sb + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
+                                           packed[4 * c + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmY, sb, n0, row0);
+                            bulk_commit();
+                        }
+                        stg_sel ^= 1;
                     } else {
+                        const int row = row0 + lane;
+                        if (row < p.M) {
+                            uint16_t* yrow = p.y + (size_t)row * p.N;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (n0 + j < p.N) yrow[n0 + j] = (uint16_t)(packed[j / 2] >> (16 * (j & 1)));
+                            for (int j = 0; j < 32; ++j)
+                                if (n0 + j < p.N) yrow[n0 + j] = (uint16_t)(packed[j / 2] >> (16 * (j & 1)));
+                        }
                     }
+                }
+                if (i == 1 && owns_overlap) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(ovl_free);
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
-            acc_phase ^= 1;
+            if (lane == 0) mbar_arrive(&acc_free[b]);
         }
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -280,7 +368,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 2-D uint8 view [rows, row_bytes] with a [box_rows, 128-byte] box, 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
+bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes,
+                      int box_rows) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
@@ -290,6 +379,20 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_byte
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// bf16 [M, N] output with a 32 x 32 box and 64-byte swizzle (N % 8 == 0).
+bool make_output_map(CUtensorMap* map, void* base, int64_t M, int64_t N) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -304,9 +407,15 @@ nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
     int* status = nullptr;
     if ((st = status_word(&status)) != NVFP4_OK) return st;
 
-    CUtensorMap mapA, mapB;
-    if (!make_map(&mapA, a, M, K / 2, BM) || !make_map(&mapB, b, N, K / 2, BN))
+    CUtensorMap mapA, mapB, mapY;
+    if (!make_operand_map(&mapA, a, M, K / 2, BM) || !make_operand_map(&mapB, b, N, K / 2, BN))
         return NVFP4_ERR_CUDA;
+    const bool tma_store = (N % 8) == 0;
+    if (tma_store) {
+        if (!make_output_map(&mapY, y, M, N)) return NVFP4_ERR_CUDA;
+    } else {
+        mapY = mapA;   // unused
+    }
 
     static bool attr_set[64] = {false};
     if (!attr_set[dev.device & 63]) {
@@ -329,12 +438,14 @@ nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
     p.k_tiles = (int)((K + 255) / 256);
     p.kchunks = (int)(K / 64);
     p.sf_row_tiles_b = (int)((N + 127) / 128);
+    p.tma_store = tma_store ? 1 : 0;
+    p.n_fast = (N <= M) ? 1 : 0;
     p.status = status;
     p.budget_ns = 4000000000ull;   // 4 s
 
     const int tiles = p.m_blocks * p.n_blocks;
     const int grid = tiles < dev.sms ? tiles : dev.sms;
-    gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(mapA, mapB, p);
+    gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(mapA, mapB, mapY, p);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 

@@ -70,60 +70,82 @@ __device__ __forceinline__ uint4 ld_plain(const uint16_t* p) {
     return *reinterpret_cast<const uint4*>(p);
 }
 
-__device__ __forceinline__ void unpack8(const uint4& w, float (&f)[8]) {
-    f[0] = bf16lo(w.x); f[1] = bf16hi(w.x);
-    f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
-    f[4] = bf16lo(w.z); f[5] = bf16hi(w.z);
-    f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
-}
 
-// One butterfly stage on a pair: (a, b) -> (a + b, a - b), each correctly rounded.
-__device__ __forceinline__ void bfly(float& a, float& b) {
-    float s = __fadd_rn(a, b);
-    float d = __fsub_rn(a, b);
+// Packed fp32 pairs (sm_100 FADD2/FMUL2): each lane of the pair is an IEEE binary32
+// operation rounded to nearest even, exactly like its scalar form.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+// a - b as one fused op: b * (-1) is exact, so the single rounding equals rn(a - b)
+// (signed zeros included).
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 word_to_f2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
+
+// One butterfly on two packed pairs: (a, b) -> (a + b, a - b) lane-wise.
+__device__ __forceinline__ void bfly2(float2& a, float2& b) {
+    const float2 s = add2(a, b);
+    const float2 d = sub2(a, b);
     a = s;
     b = d;
 }
 
-// Rotates every g-group of the unit in place (the values stay bf16 words).
+// Rotates every g-group of the unit in place (the values stay bf16 words).  Values are
+// held as pairs (2k, 2k+1) of a chunk, so the h = 1 stage works inside a pair and all
+// later stages on whole pairs.
 template <int G>
 __device__ __forceinline__ void rotate_unit(uint4 (&w)[UnitShape<G>::NCT], int h, float hscale) {
     constexpr int NCT = UnitShape<G>::NCT;
-    float f[NCT][8];
-#pragma unroll
-    for (int i = 0; i < NCT; ++i) unpack8(w[i], f[i]);
-    // stages h = 1, 2, 4 inside each chunk
+    float2 v[NCT][4];
 #pragma unroll
     for (int i = 0; i < NCT; ++i) {
-#pragma unroll
-        for (int s = 1; s < 8; s *= 2)
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if ((e & s) == 0) bfly(f[i][e], f[i][e + s]);
+        v[i][0] = word_to_f2(w[i].x);
+        v[i][1] = word_to_f2(w[i].y);
+        v[i][2] = word_to_f2(w[i].z);
+        v[i][3] = word_to_f2(w[i].w);
     }
-    // stage h = 8: chunk 2i (lane h = 0) with chunk 2i + 1 (lane h = 1)
+#pragma unroll
+    for (int i = 0; i < NCT; ++i) {
+        // h = 1: inside each pair
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float a = v[i][k].x, b = v[i][k].y;
+            v[i][k] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+        }
+        // h = 2, 4: pairs one and two apart
+        bfly2(v[i][0], v[i][1]);
+        bfly2(v[i][2], v[i][3]);
+        bfly2(v[i][0], v[i][2]);
+        bfly2(v[i][1], v[i][3]);
+    }
+    // h = 8: chunk 2i (lane h = 0) with chunk 2i + 1 (lane h = 1); the lower lane keeps
+    // v + o, the upper lane o - v, both as o + v * (+-1) with one rounding
+    const float sg = h ? -1.0f : 1.0f;
+    const float2 sgn = make_float2(sg, sg);
 #pragma unroll
     for (int i = 0; i < NCT; ++i)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            float o = __shfl_xor_sync(kFull, f[i][e], 1);
-            f[i][e] = h ? __fsub_rn(o, f[i][e]) : __fadd_rn(f[i][e], o);
+        for (int k = 0; k < 4; ++k) {
+            const float2 o = make_float2(__shfl_xor_sync(kFull, v[i][k].x, 1),
+                                         __shfl_xor_sync(kFull, v[i][k].y, 1));
+            v[i][k] = __ffma2_rn(v[i][k], sgn, o);
         }
-    // stages h = 16, 32, 64: chunk pairs two, four, eight apart = local pairs 1, 2, 4 apart
+    // h = 16, 32, 64: chunks two, four, eight apart = local chunks 1, 2, 4 apart
 #pragma unroll
     for (int s = 1; s < G / 16; s *= 2)
 #pragma unroll
         for (int i = 0; i < NCT; ++i)
             if ((i & s) == 0)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) bfly(f[i][e], f[i + s][e]);
+                for (int k = 0; k < 4; ++k) bfly2(v[i][k], v[i + s][k]);
+    const float2 hs = make_float2(hscale, hscale);
 #pragma unroll
     for (int i = 0; i < NCT; ++i) {
-        float g[8];
+        float2 g[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(f[i][e], hscale);
-        w[i] = make_uint4(bf16x2_rn(g[0], g[1]), bf16x2_rn(g[2], g[3]), bf16x2_rn(g[4], g[5]),
-                          bf16x2_rn(g[6], g[7]));
+        for (int k = 0; k < 4; ++k) g[k] = mul2(v[i][k], hs);
+        w[i] = make_uint4(bf16x2_rn(g[0].x, g[0].y), bf16x2_rn(g[1].x, g[1].y),
+                          bf16x2_rn(g[2].x, g[2].y), bf16x2_rn(g[3].x, g[3].y));
     }
 }
 
@@ -151,6 +173,7 @@ __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
     constexpr int NCT = UnitShape<G>::NCT;
     __shared__ float red[32];
     __shared__ float s_gsf;
+    __shared__ float inv_tab[128];
 
     const int lane = threadIdx.x & 31;
     const int h = lane & 1;
@@ -173,17 +196,27 @@ __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
             if (p.gsf_out) *p.gsf_out = gsf;
             if (p.alpha_out) *p.alpha_out = __fdiv_rn(1.0f, __fmul_rn(gsf, *p.gsf_w));
         }
+        // rn(gsf / s) for every non-negative finite E4M3 scale byte (0 and NaN -> 0)
+        if (threadIdx.x < 128) {
+            const float sv = f32_from_e4m3(threadIdx.x);
+            inv_tab[threadIdx.x] = (threadIdx.x == 0 || threadIdx.x == 127) ? 0.0f : __fdiv_rn(gsf, sv);
+        }
+        __syncthreads();
     }
     float tmax = 0.0f;
 
-    for (int64_t base = warp_id * 16; base < p.total_units; base += n_warps * 16) {
-        const int64_t unit = base + (lane >> 1);
-        const bool active = unit < p.total_units;
-        int64_t row = 0, u = 0;
-        if (active) {
-            row = unit / p.upr;
-            u = unit - row * p.upr;
+    // (row, u) of this lane's unit, advanced by the grid stride without dividing again
+    const int64_t stride = n_warps * 16;
+    int64_t unit = warp_id * 16 + (lane >> 1);
+    int64_t row = unit / p.upr, u = unit - (unit / p.upr) * p.upr;
+    const int64_t srow = stride / p.upr, su = stride - srow * p.upr;
+    for (int64_t base = warp_id * 16; base < p.total_units; base += stride,
+                 unit += stride, row += srow, u += su) {
+        if (u >= p.upr) {
+            u -= p.upr;
+            ++row;
         }
+        const bool active = unit < p.total_units;
         const int64_t e0 = u * E;
         const int valid = active ? (int)min((int64_t)E, p.K - e0) : 0;
         const bool data_row = active && row < p.rows;
@@ -211,25 +244,33 @@ __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
 #pragma unroll
             for (int i = 0; i < NCT; ++i) tmax = fmaxf(tmax, absmax_words4(w[i]));
         } else {
-            // block i of the unit = chunks 2i (lane h = 0) and 2i + 1 (lane h = 1)
-            uint32_t codes[NCT];
-            uint32_t s8[NCT];
+            // block i of the unit = chunks 2i (lane h = 0) and 2i + 1 (lane h = 1).  Each
+            // lane derives the scale of the blocks i with (i & 1) == h; the pair swaps them.
+            float bm[NCT];
 #pragma unroll
             for (int i = 0; i < NCT; ++i) {
                 const float tm = absmax_words4(w[i]);
-                const float bmax = fmaxf(tm, __shfl_xor_sync(kFull, tm, 1));
-                const float s_raw = __fdiv_rn(__fmul_rn(gsf, bmax), 6.0f);
-                s8[i] = e4m3_from_f32(s_raw);
-                const float s = f32_from_e4m3(s8[i]);
-                codes[i] = 0u;
-                if (s != 0.0f) {
-                    const float inv = __fdiv_rn(gsf, s);
-                    float v[8];
-                    unpack8(w[i], v);
+                bm[i] = fmaxf(tm, __shfl_xor_sync(kFull, tm, 1));
+            }
+            uint32_t s8[NCT];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(v[e], inv);
-                    codes[i] = e2m1x8_from_f32(v);
-                }
+            for (int j = 0; j < NCT / 2; ++j) {
+                const float mine_bm = h ? bm[2 * j + 1] : bm[2 * j];
+                const uint32_t mine = e4m3_from_f32(__fdiv_rn(__fmul_rn(gsf, mine_bm), 6.0f));
+                const uint32_t other = __shfl_xor_sync(kFull, mine, 1);
+                s8[2 * j] = h ? other : mine;
+                s8[2 * j + 1] = h ? mine : other;
+            }
+            uint32_t codes[NCT];
+#pragma unroll
+            for (int i = 0; i < NCT; ++i) {
+                // inv_tab[s8] = rn(gsf / dec(s8)); a zero scale zeroes the whole block
+                const float inv = inv_tab[s8[i]];
+                const float2 iv = make_float2(inv, inv);
+                const float2 a = mul2(word_to_f2(w[i].x), iv), b = mul2(word_to_f2(w[i].y), iv);
+                const float2 c = mul2(word_to_f2(w[i].z), iv), d = mul2(word_to_f2(w[i].w), iv);
+                const float q[8] = {a.x, a.y, b.x, b.y, c.x, c.y, d.x, d.y};
+                codes[i] = s8[i] ? e2m1x8_from_f32(q) : 0u;
             }
             // scale words: blocks 4q..4q+3 -> one aligned 32-bit word, lane h = q & 1
 #pragma unroll

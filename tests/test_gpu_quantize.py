@@ -67,7 +67,7 @@ def test_quantize_rotated(oracle, group, R, K, dynamic):
 
 
 def test_quantize_special_values(oracle):
-    R, K = 130, 192
+    R, K = 130, 256
     x = torch.randn(R, K, generator=torch.Generator().manual_seed(5))
     x[0] = 0                                # all-zero row
     x[1, :16] = 0                           # all-zero block
@@ -75,8 +75,12 @@ def test_quantize_special_values(oracle):
     x[3] *= 1e30                            # huge values
     x[4, 5] = -0.0
     x[5, :] = -1e-3                         # negative values rounding to zero codes
+    x[6] *= 1e-38                           # subnormal bf16 values
     xb = x.to(torch.bfloat16)
     check(oracle, xb, 0, None)
+    for g in (16, 64, 128):                 # the rotation on the same rows
+        check(oracle, xb, g, None)
+        check(oracle, xb, g, 1.0)
     check(oracle, xb, 0, 1.0)               # unit scale (the pages' probe)
     check(oracle, xb, 0, 1e6)               # static scale far too large: saturation
     check(oracle, torch.zeros(3, 64, dtype=torch.bfloat16), 0, None)
