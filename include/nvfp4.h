@@ -177,6 +177,47 @@ NVFP4_API nvfp4_status nvfp4_linear(const void* x_bf16, int64_t M, int64_t K, co
                           const void* bias_bf16, const float* gsf_x, int rotate_group,
                           void* workspace, size_t ws_bytes, void* y_bf16, void* stream);
 
+/* Size of the library's own fixed device scratch used by
+ * nvfp4_linear_fixed_scratch: 8 MiB. */
+#define NVFP4_FIXED_SCRATCH_BYTES ((size_t)8 << 20)
+
+/*
+ * nvfp4_linear_fixed_scratch -- nvfp4_linear without a caller workspace.  The
+ * pages have no counterpart: this is a convenience of the library, not a step
+ * of the method.  It computes exactly what nvfp4_linear computes (same kernels,
+ * same arguments minus the workspace).
+ *
+ * Who it is for: callers that cannot allocate device memory at call time or
+ * have none to lend -- a C host program without a device allocator of its own,
+ * a serving process that reserved all device memory up front, or a path where
+ * a cudaMalloc would synchronise the device and stall the other streams.  The
+ * call itself allocates nothing: the packed activation, its scales, the two
+ * device scalars and the amax partials live in one fixed array of
+ * NVFP4_FIXED_SCRATCH_BYTES bytes inside the library, placed in device memory
+ * when the library's module is loaded.
+ *
+ * Limit: nvfp4_linear_workspace_bytes(M, K) <= NVFP4_FIXED_SCRATCH_BYTES
+ * (for example M*K up to about 14.8 M values: 4096 x 3584, or one
+ * 4096 x 1024 tile); a larger call returns NVFP4_ERR_WORKSPACE and launches
+ * nothing.
+ *
+ * Set-up: the first call on each device (with that device current) looks up the
+ * scratch address once; make that first call before any stream capture.
+ * Nothing in the scratch has to start at zero: each call writes every scratch
+ * byte it reads before reading it.
+ *
+ * Races: the scratch is one per device, so two calls on the same device that
+ * can overlap (different streams, or different host threads without ordering)
+ * race on it and corrupt each other.  Calls on one stream are ordered and safe.
+ *
+ * Arguments, layouts, alignment and the other errors: as nvfp4_linear.
+ */
+NVFP4_API nvfp4_status nvfp4_linear_fixed_scratch(const void* x_bf16, int64_t M, int64_t K,
+                                                  const uint8_t* w_packed, const uint8_t* w_sf,
+                                                  const float* gsf_w, int64_t N,
+                                                  const void* bias_bf16, const float* gsf_x,
+                                                  int rotate_group, void* y_bf16, void* stream);
+
 /*
  * nvfp4_last_device_status -- synchronises `stream`, then returns (in *status,
  * host pointer) and clears the current device's asynchronous status word:

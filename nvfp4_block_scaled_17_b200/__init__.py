@@ -38,6 +38,8 @@ SIGNATURES = {
     "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64]),
     "nvfp4_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _int, _vp, _sz, _vp,
                             _vp]),
+    "nvfp4_linear_fixed_scratch": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _int,
+                                          _vp, _vp]),
     "nvfp4_last_device_status": (_int, [_vp, ctypes.POINTER(_int)]),
     "nvfp4_debug_cvt_sweep": (_int, [_u32, _i64, _vp, _vp, _vp]),
     "nvfp4_debug_wait_timeout": (_int, [_i64, _vp]),
@@ -189,6 +191,33 @@ def nvfp4_linear(x: torch.Tensor, w_packed: torch.Tensor, w_sf: torch.Tensor,
         _ptr(x), M, K, _ptr(w_packed), _ptr(w_sf), _ptr(gsf_w), N, _ptr(bias), _ptr(gsf_x),
         int(rotate_group), _ptr(workspace), workspace.numel(), _ptr(y), _stream(stream)))
     return y
+
+
+FIXED_SCRATCH_BYTES = 8 << 20
+
+
+def nvfp4_linear_fixed_scratch(x: torch.Tensor, w_packed: torch.Tensor, w_sf: torch.Tensor,
+                               gsf_w: torch.Tensor, N: int, out: torch.Tensor,
+                               bias: torch.Tensor | None = None,
+                               gsf_x: torch.Tensor | None = None, rotate_group: int = 0,
+                               stream=None) -> torch.Tensor:
+    """nvfp4_linear for callers that cannot hand over a workspace: the library's
+    own fixed device scratch (FIXED_SCRATCH_BYTES per device) holds the packed
+    activation.  Nothing is allocated here either, so `out` and the device
+    scalars are required as tensors.  Calls on one device that can overlap race
+    on the shared scratch; make the first call on a device before any stream
+    capture."""
+    _bf16_2d(x, "x")
+    M, K = x.shape
+    for t, name in ((gsf_w, "gsf_w"), (gsf_x, "gsf_x")):
+        if t is not None and not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a one-element CUDA float32 tensor")
+    gsf_x = _scalar(gsf_x, x.device, "gsf_x")
+    gsf_w = _scalar(gsf_w, x.device, "gsf_w")
+    _check("nvfp4_linear_fixed_scratch", lib().nvfp4_linear_fixed_scratch(
+        _ptr(x), M, K, _ptr(w_packed), _ptr(w_sf), _ptr(gsf_w), N, _ptr(bias), _ptr(gsf_x),
+        int(rotate_group), _ptr(out), _stream(stream)))
+    return out
 
 
 def pack_weight(w: torch.Tensor, rotate_group: int = 0, stream=None):

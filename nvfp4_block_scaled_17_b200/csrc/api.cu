@@ -79,6 +79,31 @@ nvfp4_status status_word(int** dev_ptr) {
     return NVFP4_OK;
 }
 
+// Fixed scratch of nvfp4_linear_fixed_scratch: one per device, placed when the
+// module loads.  Holds the same carve as a caller workspace of nvfp4_linear.
+static __device__ __align__(256) uint8_t g_fixed_scratch[NVFP4_FIXED_SCRATCH_BYTES];
+
+namespace {
+
+uint8_t* g_fixed_scratch_ptr[kMaxDevices];
+
+// Address of this device's fixed scratch; looked up once per device, with the
+// device current.
+nvfp4_status fixed_scratch(uint8_t** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_fixed_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fixed_scratch) != cudaSuccess) return NVFP4_ERR_CUDA;
+        g_fixed_scratch_ptr[dev] = static_cast<uint8_t*>(p);
+    }
+    *out = g_fixed_scratch_ptr[dev];
+    return NVFP4_OK;
+}
+}  // namespace
+
 }  // namespace nvfp4
 
 using namespace nvfp4;
@@ -193,6 +218,39 @@ nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w_
     if (M == 0 || N == 0) return NVFP4_OK;
 
     uint8_t* base = static_cast<uint8_t*>(workspace);
+    uint8_t* xp = base + ws.packed;
+    uint8_t* xsf = base + ws.sf;
+    float* scalars = reinterpret_cast<float*>(base + ws.scalars);
+    float* partials = reinterpret_cast<float*>(base + ws.partials);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_quantize(x, M, K, group, gsf_x, &scalars[0], xp, xsf, partials, gsf_w, &scalars[1],
+                         s);
+    if (st != NVFP4_OK) return st;
+    return launch_gemm(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s);
+}
+
+nvfp4_status nvfp4_linear_fixed_scratch(const void* x, int64_t M, int64_t K,
+                                        const uint8_t* w_packed, const uint8_t* w_sf,
+                                        const float* gsf_w, int64_t N, const void* bias,
+                                        const float* gsf_x, int group, void* y, void* stream) {
+    if (!x || !w_packed || !w_sf || !gsf_w || !y || M < 0 || N < 0 || !valid_group(group))
+        return NVFP4_ERR_INVALID_ARG;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 64 || (group && K % group) || K >= (int64_t(1) << 31))
+        return NVFP4_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(w_packed, 16) || !aligned(w_sf, 16) || !aligned(y, 16) ||
+        !aligned(gsf_w, 4) || (gsf_x && !aligned(gsf_x, 4)) || (bias && !aligned(bias, 16)))
+        return NVFP4_ERR_ALIGN;
+    const LinearWs ws = linear_ws(M, K);
+    if (ws.total > NVFP4_FIXED_SCRATCH_BYTES) return NVFP4_ERR_WORKSPACE;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    uint8_t* base = nullptr;
+    st = fixed_scratch(&base);
+    if (st != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return NVFP4_OK;
+
     uint8_t* xp = base + ws.packed;
     uint8_t* xsf = base + ws.sf;
     float* scalars = reinterpret_cast<float*>(base + ws.scalars);

@@ -82,6 +82,10 @@ def test_gemm_and_linear_argument_errors(L):
     assert lin(A, 4, 96, A, A, A, 8, None, None, 0, A, 1 << 20, A, S) == nv.ERR_SHAPE
     assert lin(A, 4, 128, A, A, A, 8, None, None, 48, A, 1 << 20, A, S) == nv.ERR_INVALID_ARG
     assert lin(A, 4, 128, A, A, None, 8, None, None, 0, A, 1 << 20, A, S) == nv.ERR_INVALID_ARG
+    fx = L.nvfp4_linear_fixed_scratch
+    assert fx(A, 16384, 1024, A, A, A, 8, None, None, 0, A, S) == nv.ERR_WORKSPACE  # > 8 MiB
+    assert fx(A, 4, 96, A, A, A, 8, None, None, 0, A, S) == nv.ERR_SHAPE
+    assert fx(A, 4, 128, A, A, None, 8, None, None, 0, A, S) == nv.ERR_INVALID_ARG
     h = L.hadamard_rotate
     assert h(A, A, 4, 64, 0, S) == nv.ERR_INVALID_ARG
     assert h(A, A, 4, 96, 64, S) == nv.ERR_SHAPE
