@@ -65,6 +65,7 @@ def measured_traffic(key):
 GROUP = 128
 TOKENS = 8 * 4096
 CPU_SAMPLE_ROWS = 768
+REF_SAMPLE_ROWS = 64
 
 
 def peaks():
@@ -224,11 +225,24 @@ def timed_steps(layers, dynamic, steps, warmup, dist_on):
 
 
 def max_over_ranks(v: float, dist_on: bool) -> float:
+    """The slowest rank's figure (a device tensor under NCCL, a host one under gloo)."""
     if not dist_on:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_tflops(flops_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job throughput under weak scaling: every rank processes its own batch of
+    the same size, so the job does world x the per-rank work in the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own independent batch."""
+    return 1001 + rank
 
 
 def e2e_steps(layers, steps, warmup, dist_on):
@@ -286,17 +300,29 @@ def weight_pack_rate(layers_src, dev):
             "bytes_per_value": 8.5625}
 
 
-def cpu_baseline(layers_src, rows: int):
-    """The oracle as it stands on the host cores: rotate, dynamic quantize and the fp64
-    GEMM for `rows` rows of each linear (weights packed by the oracle, untimed)."""
-    import numpy as np
-
+def oracle_pack(layers_src):
+    """The oracle's own weight packing (rotate g=128, dynamic quantize); untimed."""
     import oracle as O
     O.build()
-    packed = []
-    for l in layers_src:
-        wr = O.hadamard_rotate(W.to_u16(l.weight), GROUP)
-        packed.append(O.quantize(wr))
+    return [O.quantize(O.hadamard_rotate(W.to_u16(l.weight), GROUP)) for l in layers_src]
+
+
+def host_cores() -> int:
+    n = os.environ.get("OMP_NUM_THREADS")
+    if n:
+        return int(n)
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(layers_src, rows: int, packed=None):
+    """The oracle as it stands on the host cores: rotate, dynamic quantize and the fp64
+    GEMM for `rows` rows of each linear (weights packed by the oracle, untimed)."""
+    import oracle as O
+    if packed is None:
+        packed = oracle_pack(layers_src)
     xs = [W.to_u16(l.x[:rows]) for l in layers_src]
     bs = [W.to_u16(l.bias) for l in layers_src]
     t0 = time.perf_counter()
@@ -305,8 +331,8 @@ def cpu_baseline(layers_src, rows: int):
         O.linear(x, wp, wsf, gw, l.N, b, rotate_group=GROUP)
         flops += 2.0 * rows * l.N * l.K
     dt = time.perf_counter() - t0
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(),
+            "kind": "oracle",
             "sample": f"{rows} rows of each of the 4 linears (rotate g=128, dynamic quantize, "
                       f"fp64 GEMM over all N), {dt:.1f} s"}, dt
 
@@ -317,7 +343,7 @@ def run_ours(args, dist_on, rank, world, local_rank):
     props = torch.cuda.get_device_properties(dev)
     l2 = int(getattr(props, "L2_cache_size", 126 * 1024 * 1024))
     pk = peaks()
-    src = W.vit_block(dev, seed=1001 + rank, tokens=TOKENS)
+    src = W.vit_block(dev, seed=rank_seed(rank), tokens=TOKENS)
     layers = [Layer(l, dev) for l in src]
     # static scale: the scale a calibration pass over this very input would store, i.e.
     # the dynamic scale of one untimed call
@@ -344,7 +370,7 @@ def run_ours(args, dist_on, rank, world, local_rank):
     ms = max_over_ranks(total_ms / args.steps, dist_on)
     s_ms = max_over_ranks(s_total / args.steps, dist_on)
     flops = sum(ly.flops() for ly in layers)
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = aggregate_tflops(flops, ms, world)
 
     fp4_peak = 4.0 * pk["bf16_sus"]           # nominal fp4 / bf16 = 9 / 2.25
     g_time = sum(g_ms)
@@ -376,10 +402,10 @@ def run_ours(args, dist_on, rank, world, local_rank):
         "config": workload_config("dynamic"),
         "roofline": gemm_roof if dominant_is_gemm else quant_roof,
         "roofline_gemm": gemm_roof, "roofline_quantizer": quant_roof,
-        "static_scale": {"ms_per_step": s_ms, "TFLOP/s": world * flops / (s_ms * 1e-3) / 1e12,
+        "static_scale": {"ms_per_step": s_ms, "TFLOP/s": aggregate_tflops(flops, s_ms, world),
                          "quantizer_ms": s_q, "gemm_ms": s_g},
         "weight_pack": wpack,
-        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": aggregate_tflops(flops, e2e_ms, world), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "nvfp4_linear"},
         "gpu_launches": 3 * len(layers) * args.steps,
@@ -393,19 +419,23 @@ def run_ours(args, dist_on, rank, world, local_rank):
 
 def run_reference(args, rank, world):
     """The oracle as the reference arm: each step is a bounded sample of the same
-    workload (rows of each linear) on the host cores; rank 0 only."""
+    workload (REF_SAMPLE_ROWS rows of each linear, about 1-2 s on the host cores);
+    rank 0 only, the other ranks exit without work."""
     if rank != 0:
         return None
-    src = W.vit_block("cpu", seed=1001, tokens=CPU_SAMPLE_ROWS)
+    src = W.vit_block("cpu", seed=1001, tokens=REF_SAMPLE_ROWS)
+    packed = oracle_pack(src)
     for _ in range(args.warmup):
-        cpu_baseline(src, 32)
+        cpu_baseline(src, 8, packed)
     vals, dts = [], []
     for _ in range(args.steps):
-        cb, dt = cpu_baseline(src, CPU_SAMPLE_ROWS // 4)
+        cb, dt = cpu_baseline(src, REF_SAMPLE_ROWS, packed)
         vals.append(cb["value"])
         dts.append(dt)
-    v = statistics.mean(vals)
+    v = sum(2.0 * REF_SAMPLE_ROWS * l.N * l.K for l in src) * len(dts) / sum(dts) / 1e12
     cb["value"] = v
+    cb["sample"] = (f"{REF_SAMPLE_ROWS} rows of each of the 4 linears per step (rotate g=128, "
+                    f"dynamic quantize, fp64 GEMM over all N), {args.steps} steps")
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(dts),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
