@@ -24,7 +24,8 @@
  *     device, owned by the caller.  The library never allocates, frees or
  *     synchronises (except nvfp4_last_device_status, which says so); each call only
  *     enqueues kernels on `stream` (a cudaStream_t; NULL = legacy default stream),
- *     so calls are stream-ordered and may be captured in a CUDA graph.
+ *     so calls are stream-ordered and may be captured in a CUDA graph
+ *     (nvfp4_linear_fixed_scratch states its own set-up condition).
  *   - bf16 tensors are row-major with no padding; tensor pointers must be 16-byte
  *     aligned, scalar pointers 4-byte aligned.
  *   - Argument checks run on the host before anything is enqueued; on any error
@@ -231,12 +232,14 @@ NVFP4_API nvfp4_status nvfp4_last_device_status(void* stream, int* status);
 /*
  * nvfp4_debug_cvt_sweep -- runs the quantizer's own device conversions over the
  * fp32 bit patterns first, first+1, ..., first+n-1 (wrapping mod 2^32):
- *   e2m1[i] = E2M1 code of the pattern (RNE, saturating, sign kept)
- *   e4m3[i] = E4M3 byte of |pattern| (RNE, saturating)
- * Both outputs: device uint8 [n].  Errors: INVALID_ARG, DEVICE, CUDA.
+ *   e2m1[i]  = E2M1 code of the pattern (RNE, saturating, sign kept)
+ *   e4m3[i]  = E4M3 byte of |pattern| (RNE, saturating)
+ *   scale[i] = the block-scale byte the quantizer derives from a scaled block
+ *              maximum y = |pattern|: E4M3(rn(y / 6))
+ * All outputs: device uint8 [n].  Errors: INVALID_ARG, DEVICE, CUDA.
  */
 NVFP4_API nvfp4_status nvfp4_debug_cvt_sweep(uint32_t first, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
-                                   void* stream);
+                                             uint8_t* scale, void* stream);
 
 /*
  * nvfp4_debug_wait_timeout -- launches one block that waits on a barrier nothing

@@ -41,7 +41,7 @@ SIGNATURES = {
     "nvfp4_linear_fixed_scratch": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _int,
                                           _vp, _vp]),
     "nvfp4_last_device_status": (_int, [_vp, ctypes.POINTER(_int)]),
-    "nvfp4_debug_cvt_sweep": (_int, [_u32, _i64, _vp, _vp, _vp]),
+    "nvfp4_debug_cvt_sweep": (_int, [_u32, _i64, _vp, _vp, _vp, _vp]),
     "nvfp4_debug_wait_timeout": (_int, [_i64, _vp]),
 }
 

@@ -65,6 +65,20 @@ nvfp4_status device_info(DeviceInfo* out) {
     return NVFP4_OK;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
 nvfp4_status status_word(int** dev_ptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -279,13 +293,13 @@ nvfp4_status nvfp4_last_device_status(void* stream, int* status) {
 }
 
 nvfp4_status nvfp4_debug_cvt_sweep(uint32_t first, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
-                                   void* stream) {
-    if (!e2m1 || !e4m3 || n < 0 || n > (int64_t(1) << 32)) return NVFP4_ERR_INVALID_ARG;
+                                   uint8_t* scale, void* stream) {
+    if (!e2m1 || !e4m3 || !scale || n < 0 || n > (int64_t(1) << 32)) return NVFP4_ERR_INVALID_ARG;
     DeviceInfo dev;
     nvfp4_status st = device_info(&dev);
     if (st != NVFP4_OK) return st;
     if (n == 0) return NVFP4_OK;
-    return launch_cvt_sweep(first, n, e2m1, e4m3, static_cast<cudaStream_t>(stream));
+    return launch_cvt_sweep(first, n, e2m1, e4m3, scale, static_cast<cudaStream_t>(stream));
 }
 
 nvfp4_status nvfp4_debug_wait_timeout(int64_t budget_us, void* stream) {

@@ -33,6 +33,21 @@ __device__ __forceinline__ uint32_t e4m3_from_f32(float v) {
     return r & 0xffu;
 }
 
+// Block-scale byte of a block whose scaled maximum is y = rn(gsf * bmax) >= 0:
+// E4M3(rn(y / 6)), with the quotient rounded correctly without a divide instruction.
+// With r = rn(1/6) (within half an ulp of 1/6) the first quotient q0 = rn(y * r) is
+// faithful, the remainder y - 6 * q0 is then exact in one FMA, and q0 + rem * r rounded
+// once is rn(y / 6): the correction step of Markstein's division theorem.  y above
+// 6000 is clamped first (every y / 6 >= 448 saturates to the same byte, and the clamp
+// keeps the remainder finite); NaN passes through to the NaN byte as before.
+__device__ __forceinline__ uint32_t e4m3_scale_of_scaled_max(float y) {
+    const float r = __uint_as_float(0x3e2aaaabu);   // rn(1/6)
+    y = (y > 6000.0f) ? 6000.0f : y;
+    const float q0 = __fmul_rn(y, r);
+    const float rem = __fmaf_rn(-q0, 6.0f, y);
+    return e4m3_from_f32(__fmaf_rn(rem, r, q0));
+}
+
 // fp32 value of an E4M3 byte (exact: E4M3 -> f16 -> f32 are both widening).
 __device__ __forceinline__ float f32_from_e4m3(uint32_t b) {
     uint32_t h2;
@@ -80,18 +95,26 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// max(|lo|, |hi|) of a bf16 pair, as bf16 bits in the low half.  The max of the
-// magnitudes is exact in any order.
-__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
-    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
-    __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
-    __nv_bfloat162 m = __hmax2(__habs2(x), __habs2(y));
-    return *reinterpret_cast<uint32_t*>(&m);
+// Lane-wise max(|a|, |b|) of two bf16 pairs.  The magnitudes are exact; the sign
+// bits of the result are not meaningful (callers take magnitudes).
+__device__ __forceinline__ uint32_t absmax2_bf16(uint32_t a, uint32_t b) {
+    uint32_t m;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(a), "r"(b));
+    return m;
+}
+
+// Both magnitudes of the largest-|.| pair of four bf16 pairs (one 8-value chunk).
+__device__ __forceinline__ uint32_t absmax_word4(const uint4& w) {
+    return absmax2_bf16(absmax2_bf16(w.x, w.y), absmax2_bf16(w.z, w.w));
+}
+
+// The larger magnitude of a bf16 pair as a float.
+__device__ __forceinline__ float absmax_of_pair(uint32_t m) {
+    return fmaxf(fabsf(__uint_as_float(m << 16)), fabsf(__uint_as_float(m & 0xffff0000u)));
 }
 
 __device__ __forceinline__ float absmax_words4(const uint4& w) {
-    uint32_t m = absmax_bf16x2(absmax_bf16x2(w.x, w.y), absmax_bf16x2(w.z, w.w));
-    return fmaxf(bf16lo(m), bf16hi(m));
+    return absmax_of_pair(absmax_word4(w));
 }
 
 // ---------------------------------------------------------------------------
@@ -178,6 +201,28 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
+}
+
+// The same load with an L2 eviction-priority policy (from l2_policy_*).
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int32_t x, int32_t y, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+// L2 policies: keep lines that will be read again soon, or let read-once lines go first.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,

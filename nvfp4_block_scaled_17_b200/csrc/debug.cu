@@ -11,12 +11,14 @@ namespace nvfp4 {
 
 namespace {
 
-__global__ void cvt_sweep_kernel(uint32_t first, int64_t n, uint8_t* e2m1, uint8_t* e4m3) {
+__global__ void cvt_sweep_kernel(uint32_t first, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
+                                 uint8_t* scale) {
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
         const float v = __uint_as_float(first + (uint32_t)i);
         e2m1[i] = (uint8_t)(e2m1x2_from_f32(v, 0.0f) & 0xfu);
         e4m3[i] = (uint8_t)e4m3_from_f32(fabsf(v));
+        scale[i] = (uint8_t)e4m3_scale_of_scaled_max(fabsf(v));
     }
 }
 
@@ -39,13 +41,13 @@ __global__ void wait_timeout_kernel(uint64_t budget_ns, int* status) {
 }  // namespace
 
 nvfp4_status launch_cvt_sweep(uint32_t first, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
-                              cudaStream_t stream) {
+                              uint8_t* scale, cudaStream_t stream) {
     DeviceInfo dev;
     nvfp4_status st = device_info(&dev);
     if (st != NVFP4_OK) return st;
     int64_t blocks = (n + 255) / 256;
     const int grid = (int)(blocks < dev.sms * 16 ? blocks : dev.sms * 16);
-    cvt_sweep_kernel<<<grid, 256, 0, stream>>>(first, n, e2m1, e4m3);
+    cvt_sweep_kernel<<<grid, 256, 0, stream>>>(first, n, e2m1, e4m3, scale);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 

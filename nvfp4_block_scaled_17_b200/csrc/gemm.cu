@@ -269,78 +269,90 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             const bool owns_overlap = (b == 0) ? (half == 1) : (half == 0);
             const uint32_t buf_col = b ? TMEM_BUF1 : 0u;
             const int row0 = m_blk * BM + quad * 32;
-            for (int i = 0; i < 4; ++i) {
-                const int chunk = (b == 0 && half == 1) ? ((i + 2) & 3) + 4 : half * 4 + i;
+            // bf16(alpha * acc + bias) of one 32-column chunk, staged and stored
+            auto store_chunk = [&](const uint32_t (&r)[32], int chunk) {
                 const int n0 = n_blk * BN + chunk * 32;
-                if (n0 < p.N) {   // warp-uniform
-                    uint32_t r[32];
-                    tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + buf_col + (uint32_t)chunk * 32, r);
-                    tmem_ld_wait();
-                    float bv[32];
-                    if (p.bias) {
-                        if (n0 + 32 <= p.N) {
-                            const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0);
+                if (n0 >= p.N) return;   // warp-uniform
+                float bv[32];
+                if (p.bias) {
+                    if (n0 + 32 <= p.N) {
+                        const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0);
 #pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4) {
-                                const uint4 w = bp[q4];
-                                bv[8 * q4 + 0] = bf16lo(w.x); bv[8 * q4 + 1] = bf16hi(w.x);
-                                bv[8 * q4 + 2] = bf16lo(w.y); bv[8 * q4 + 3] = bf16hi(w.y);
-                                bv[8 * q4 + 4] = bf16lo(w.z); bv[8 * q4 + 5] = bf16hi(w.z);
-                                bv[8 * q4 + 6] = bf16lo(w.w); bv[8 * q4 + 7] = bf16hi(w.w);
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                bv[j] = __uint_as_float((uint32_t)p.bias[min(n0 + j, p.N - 1)] << 16);
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const uint4 w = bp[q4];
+                            bv[8 * q4 + 0] = bf16lo(w.x); bv[8 * q4 + 1] = bf16hi(w.x);
+                            bv[8 * q4 + 2] = bf16lo(w.y); bv[8 * q4 + 3] = bf16hi(w.y);
+                            bv[8 * q4 + 4] = bf16lo(w.z); bv[8 * q4 + 5] = bf16hi(w.z);
+                            bv[8 * q4 + 6] = bf16lo(w.w); bv[8 * q4 + 7] = bf16hi(w.w);
                         }
-                    }
-                    uint32_t packed[16];
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        float v0 = __fmul_rn(alpha, __uint_as_float(r[j]));
-                        float v1 = __fmul_rn(alpha, __uint_as_float(r[j + 1]));
-                        if (p.bias) {
-                            v0 = __fadd_rn(v0, bv[j]);
-                            v1 = __fadd_rn(v1, bv[j + 1]);
-                        }
-                        packed[j / 2] = bf16x2_bits(v0, v1);
-                    }
-                    if (p.tma_store) {
-                        uint8_t* sb = stg + stg_sel * STG_BYTES;
-                        if (lane == 0) bulk_wait_read<1>();   // this buffer's previous store
-                        __syncwarp();
-                        // 64-byte swizzle: 16-byte chunk c of row r sits at c ^ ((r >> 1) & 3)
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            *reinterpret_cast<uint4*>(sb + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
-                                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
-                                           packed[4 * c + 3]);
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&tmY, sb, n0, row0);
-                            bulk_commit();
-                        }
-                        stg_sel ^= 1;
                     } else {
-                        const int row = row0 + lane;
-                        if (row < p.M) {
-                            uint16_t* yrow = p.y + (size_t)row * p.N;
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (n0 + j < p.N) yrow[n0 + j] = (uint16_t)(packed[j / 2] >> (16 * (j & 1)));
-                        }
+                        for (int j = 0; j < 32; ++j)
+                            bv[j] = __uint_as_float((uint32_t)p.bias[min(n0 + j, p.N - 1)] << 16);
                     }
                 }
-                if (i == 1 && owns_overlap) {
+                uint32_t packed[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    float v0 = __fmul_rn(alpha, __uint_as_float(r[j]));
+                    float v1 = __fmul_rn(alpha, __uint_as_float(r[j + 1]));
+                    if (p.bias) {
+                        v0 = __fadd_rn(v0, bv[j]);
+                        v1 = __fadd_rn(v1, bv[j + 1]);
+                    }
+                    packed[j / 2] = bf16x2_bits(v0, v1);
+                }
+                if (p.tma_store) {
+                    uint8_t* sb = stg + stg_sel * STG_BYTES;
+                    if (lane == 0) bulk_wait_read<1>();   // this buffer's previous store
+                    __syncwarp();
+                    // 64-byte swizzle: 16-byte chunk c of row r sits at c ^ ((r >> 1) & 3)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(sb + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
+                                       packed[4 * c + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmY, sb, n0, row0);
+                        bulk_commit();
+                    }
+                    stg_sel ^= 1;
+                } else {
+                    const int row = row0 + lane;
+                    if (row < p.M) {
+                        uint16_t* yrow = p.y + (size_t)row * p.N;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (n0 + j < p.N) yrow[n0 + j] = (uint16_t)(packed[j / 2] >> (16 * (j & 1)));
+                    }
+                }
+            };
+            // Two chunks at a time: both tensor-memory loads are in flight together, and
+            // the columns are released as soon as they are in registers -- the shared
+            // columns first, so the next tile's MMAs start before this tile is stored.
+            const uint32_t lane_col = tmem + ((uint32_t)(quad * 32) << 16) + buf_col;
+            for (int i = 0; i < 4; i += 2) {
+                const int c0 = (b == 0 && half == 1) ? ((i + 2) & 3) + 4 : half * 4 + i;
+                const int c1 = (b == 0 && half == 1) ? ((i + 3) & 3) + 4 : half * 4 + i + 1;
+                uint32_t r0[32], r1[32];
+                tmem_ld32(lane_col + (uint32_t)c0 * 32, r0);
+                tmem_ld32(lane_col + (uint32_t)c1 * 32, r1);
+                tmem_ld_wait();
+                if (i == 0 && owns_overlap) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(ovl_free);
                 }
+                if (i == 2) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_free[b]);
+                }
+                store_chunk(r0, c0);
+                store_chunk(r1, c1);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_free[b]);
         }
         if (lane == 0) bulk_wait_all();
         __syncwarp();
@@ -352,19 +364,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
-                                             cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
 }
 
 // 2-D uint8 view [rows, row_bytes] with a [box_rows, 128-byte] box, 128-byte swizzle.

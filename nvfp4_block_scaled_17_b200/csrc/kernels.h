@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 
 #include "nvfp4.h"
@@ -35,8 +36,12 @@ nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          int64_t M, int64_t N, int64_t K, cudaStream_t stream);
 
 nvfp4_status launch_cvt_sweep(uint32_t first, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
-                              cudaStream_t stream);
+                              uint8_t* scale, cudaStream_t stream);
 nvfp4_status launch_wait_timeout(int64_t budget_us, cudaStream_t stream);
+
+// The driver's cuTensorMapEncodeTiled (looked up once through the runtime), or
+// nullptr when the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // The per-device asynchronous status word (device address for the current device).
 nvfp4_status status_word(int** dev_ptr);

@@ -93,25 +93,32 @@ __device__ __forceinline__ void bfly2(float2& a, float2& b) {
 // Rotates every g-group of the unit in place (the values stay bf16 words).  Values are
 // held as pairs (2k, 2k+1) of a chunk, so the h = 1 stage works inside a pair and all
 // later stages on whole pairs.
+// rn(lo + hi) and rn(lo - hi) of one bf16 pair, with hi widened to fp32 and lo used
+// as a bf16 operand of the mixed-precision add and subtract (exact widening, one
+// rounding each, so both equal the plain fp32 results, signed zeros included).
+__device__ __forceinline__ float2 pair_sum_diff(uint32_t w) {
+    const float hi = bf16hi(w);
+    const uint16_t lo = (uint16_t)(w & 0xffffu);
+    float s, d;
+    asm("add.rn.f32.bf16 %0, %1, %2;" : "=f"(s) : "h"(lo), "f"(hi));
+    asm("sub.rn.f32.bf16 %0, %1, %2;" : "=f"(d) : "h"(lo), "f"(hi));
+    return make_float2(s, d);
+}
+
+// Rotates every g-group of the unit in place (the values stay bf16 words).  Values are
+// held as pairs (2k, 2k+1) of a chunk, so the h = 1 stage works inside a pair and all
+// later stages on whole pairs.
 template <int G>
 __device__ __forceinline__ void rotate_unit(uint4 (&w)[UnitShape<G>::NCT], int h, float hscale) {
     constexpr int NCT = UnitShape<G>::NCT;
     float2 v[NCT][4];
 #pragma unroll
     for (int i = 0; i < NCT; ++i) {
-        v[i][0] = word_to_f2(w[i].x);
-        v[i][1] = word_to_f2(w[i].y);
-        v[i][2] = word_to_f2(w[i].z);
-        v[i][3] = word_to_f2(w[i].w);
-    }
-#pragma unroll
-    for (int i = 0; i < NCT; ++i) {
-        // h = 1: inside each pair
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float a = v[i][k].x, b = v[i][k].y;
-            v[i][k] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
-        }
+        // h = 1: inside each pair, straight from the bf16 words
+        v[i][0] = pair_sum_diff(w[i].x);
+        v[i][1] = pair_sum_diff(w[i].y);
+        v[i][2] = pair_sum_diff(w[i].z);
+        v[i][3] = pair_sum_diff(w[i].w);
         // h = 2, 4: pairs one and two apart
         bfly2(v[i][0], v[i][1]);
         bfly2(v[i][2], v[i][3]);
@@ -166,6 +173,115 @@ __device__ __forceinline__ float block_max(float v, float* red) {
     return v;   // valid in warp 0
 }
 
+// Encode-pass prologue of every CTA: the global scale (given, or reduced from the
+// amax partials: FP4_E4M3_RANGE / max(amax, floor)), alpha and gsf written once by
+// block 0, and the table rn(gsf / dec(s)) for every non-negative E4M3 scale byte
+// (0 and NaN map to 0).  Ends with a block barrier.
+template <int THREADS>
+__device__ __forceinline__ float encode_prologue(const UnitParams& p, float* red, float* s_gsf,
+                                                 float* inv_tab) {
+    float gsf;
+    if (p.gsf_in != nullptr) {
+        gsf = *p.gsf_in;
+    } else {
+        float m = 0.0f;
+        for (int i = threadIdx.x; i < p.n_partials; i += THREADS) m = fmaxf(m, p.partials[i]);
+        m = block_max(m, red);
+        if (threadIdx.x == 0) *s_gsf = __fdiv_rn(kFp4E4m3Range, fmaxf(m, kAmaxFloor));
+        __syncthreads();
+        gsf = *s_gsf;
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (p.gsf_out) *p.gsf_out = gsf;
+        if (p.alpha_out) *p.alpha_out = __fdiv_rn(1.0f, __fmul_rn(gsf, *p.gsf_w));
+    }
+    if (threadIdx.x < 128) {
+        const float sv = f32_from_e4m3(threadIdx.x);
+        inv_tab[threadIdx.x] = (threadIdx.x == 0 || threadIdx.x == 127) ? 0.0f : __fdiv_rn(gsf, sv);
+    }
+    __syncthreads();
+    return gsf;
+}
+
+// Encode pass of one unit: block maxima, E4M3 scales, E2M1 codes; writes the
+// packed bytes (rows < p.rows only) and the scale words of the 128x4 layout.
+template <int G>
+__device__ __forceinline__ void encode_unit(const uint4 (&w)[UnitShape<G>::NCT], int h, float gsf,
+                                            const float* inv_tab, const UnitParams& p,
+                                            int64_t row, int64_t e0, int valid, bool data_row,
+                                            bool active) {
+    constexpr int NCT = UnitShape<G>::NCT;
+    // block i of the unit = chunks 2i (lane h = 0) and 2i + 1 (lane h = 1).  Each
+    // lane derives the scale of the blocks i with (i & 1) == h; the pair swaps them.
+    float bm[NCT];
+#pragma unroll
+    for (int i = 0; i < NCT; ++i) {
+        const uint32_t tm = absmax_word4(w[i]);
+        bm[i] = absmax_of_pair(absmax2_bf16(tm, __shfl_xor_sync(kFull, tm, 1)));
+    }
+    uint32_t s8[NCT];
+#pragma unroll
+    for (int j = 0; j < NCT / 2; ++j) {
+        const float mine_bm = h ? bm[2 * j + 1] : bm[2 * j];
+        const uint32_t mine = e4m3_scale_of_scaled_max(__fmul_rn(gsf, mine_bm));
+        const uint32_t other = __shfl_xor_sync(kFull, mine, 1);
+        s8[2 * j] = h ? other : mine;
+        s8[2 * j + 1] = h ? mine : other;
+    }
+    uint32_t codes[NCT];
+#pragma unroll
+    for (int i = 0; i < NCT; ++i) {
+        // inv_tab[s8] = rn(gsf / dec(s8)); a zero scale zeroes the whole block
+        const float inv = inv_tab[s8[i]];
+        const float2 iv = make_float2(inv, inv);
+        const float2 a = mul2(word_to_f2(w[i].x), iv), b = mul2(word_to_f2(w[i].y), iv);
+        const float2 c = mul2(word_to_f2(w[i].z), iv), d = mul2(word_to_f2(w[i].w), iv);
+        const float q[8] = {a.x, a.y, b.x, b.y, c.x, c.y, d.x, d.y};
+        codes[i] = s8[i] ? e2m1x8_from_f32(q) : 0u;
+    }
+    // scale words: blocks 4q..4q+3 -> one aligned 32-bit word, lane h = q & 1
+#pragma unroll
+    for (int q = 0; q < NCT / 4; ++q) {
+        if (active && (q & 1) == h) {
+            const uint32_t word = s8[4 * q] | (s8[4 * q + 1] << 8) | (s8[4 * q + 2] << 16) |
+                                  (s8[4 * q + 3] << 24);
+            const int64_t cg = e0 / 64 + q;
+            const int64_t off = (((row >> 7) * p.cgroups + cg) << 9) + ((row & 31) << 4) +
+                                (((row >> 5) & 3) << 2);
+            *reinterpret_cast<uint32_t*>(p.sf + off) = word;
+        }
+    }
+    // packed bytes: each lane of the pair writes 16 contiguous bytes per 8-word half
+    const int valid_words = valid / 8;
+    uint8_t* dst = p.packed + row * (p.K / 2) + e0 / 2;
+    const bool al16 = ((row * (p.K / 2)) & 15) == 0;
+#pragma unroll
+    for (int hh = 0; hh < NCT / 4; ++hh) {
+        const uint32_t c0 = codes[4 * hh], c1 = codes[4 * hh + 1];
+        const uint32_t c2 = codes[4 * hh + 2], c3 = codes[4 * hh + 3];
+        const uint32_t r0 = __shfl_xor_sync(kFull, h ? c0 : c2, 1);
+        const uint32_t r1 = __shfl_xor_sync(kFull, h ? c1 : c3, 1);
+        const uint4 out = h ? make_uint4(r0, c2, r1, c3) : make_uint4(c0, r0, c1, r1);
+        const int wb = 8 * hh + 4 * h;
+        uint32_t* d = reinterpret_cast<uint32_t*>(dst + wb * 4);
+        if (data_row) {
+            if (wb + 4 <= valid_words) {
+                if (al16) {
+                    *reinterpret_cast<uint4*>(d) = out;
+                } else {
+                    reinterpret_cast<uint2*>(d)[0] = make_uint2(out.x, out.y);
+                    reinterpret_cast<uint2*>(d)[1] = make_uint2(out.z, out.w);
+                }
+            } else {
+                const uint32_t o[4] = {out.x, out.y, out.z, out.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (wb + j < valid_words) d[j] = o[j];
+            }
+        }
+    }
+}
+
 // MODE 0: amax partials.  MODE 1: quantize.  MODE 2: rotate only (G > 0).
 template <int G, int MODE>
 __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
@@ -181,29 +297,8 @@ __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
     const int64_t n_warps = (int64_t)gridDim.x * (kThreads / 32);
 
     float gsf = 0.0f;
-    if constexpr (MODE == 1) {
-        if (p.gsf_in != nullptr) {
-            gsf = *p.gsf_in;
-        } else {
-            float m = 0.0f;
-            for (int i = threadIdx.x; i < p.n_partials; i += kThreads) m = fmaxf(m, p.partials[i]);
-            m = block_max(m, red);
-            if (threadIdx.x == 0) s_gsf = __fdiv_rn(kFp4E4m3Range, fmaxf(m, kAmaxFloor));
-            __syncthreads();
-            gsf = s_gsf;
-        }
-        if (blockIdx.x == 0 && threadIdx.x == 0) {
-            if (p.gsf_out) *p.gsf_out = gsf;
-            if (p.alpha_out) *p.alpha_out = __fdiv_rn(1.0f, __fmul_rn(gsf, *p.gsf_w));
-        }
-        // rn(gsf / s) for every non-negative finite E4M3 scale byte (0 and NaN -> 0)
-        if (threadIdx.x < 128) {
-            const float sv = f32_from_e4m3(threadIdx.x);
-            inv_tab[threadIdx.x] = (threadIdx.x == 0 || threadIdx.x == 127) ? 0.0f : __fdiv_rn(gsf, sv);
-        }
-        __syncthreads();
-    }
-    float tmax = 0.0f;
+    if constexpr (MODE == 1) gsf = encode_prologue<kThreads>(p, red, &s_gsf, inv_tab);
+    uint32_t tmax = 0u;
 
     // (row, u) of this lane's unit, advanced by the grid stride without dividing again
     const int64_t stride = n_warps * 16;
@@ -242,82 +337,198 @@ __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
             }
         } else if constexpr (MODE == 0) {
 #pragma unroll
-            for (int i = 0; i < NCT; ++i) tmax = fmaxf(tmax, absmax_words4(w[i]));
+            for (int i = 0; i < NCT; ++i) tmax = absmax2_bf16(tmax, absmax_word4(w[i]));
         } else {
-            // block i of the unit = chunks 2i (lane h = 0) and 2i + 1 (lane h = 1).  Each
-            // lane derives the scale of the blocks i with (i & 1) == h; the pair swaps them.
-            float bm[NCT];
+            encode_unit<G>(w, h, gsf, inv_tab, p, row, e0, valid, data_row, active);
+        }
+    }
+    if constexpr (MODE == 0) {
+        const float m = block_max(absmax_of_pair(tmax), red);
+        if (threadIdx.x == 0) p.partials_out[blockIdx.x] = m;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// TMA-fed form (K % 64 == 0): the same per-unit arithmetic, with x staged in
+// shared memory by the tensor-memory accelerator.
+//
+// x is viewed as a flat 2-D array of 64-value rows (128 bytes each); an item is
+// the 16 units one warp handles (16 or 32 flat rows), loaded as one box with the
+// 128-byte swizzle, so the lane-pair reads below hit 8 distinct 16-byte bank
+// groups per quarter-warp.  Every warp keeps its own ring of kSlots items and
+// issues the load of item k + kSlots as soon as it has read item k into
+// registers, so HBM latency overlaps the arithmetic of the items in between.
+// One CTA of 16 warps per SM, persistent over the items.
+// ---------------------------------------------------------------------------
+
+constexpr int kTmaWarps = 16;
+constexpr int kTmaThreads = kTmaWarps * 32;
+constexpr int kSlots = 3;
+constexpr int kItemRows = 32;                       // flat 64-value rows per item (4 KiB)
+constexpr uint64_t kTmaWaitBudgetNs = 2000000000ull;
+
+template <int G>
+struct TmaShape {
+    static constexpr int E = UnitShape<G>::E;
+    static constexpr int SUBS = 128 / E;                // units per lane pair per item
+    static constexpr int UPI = 16 * SUBS;               // units per item
+    static constexpr int ITEM_BYTES = kItemRows * 128;
+    static constexpr int RING_BYTES = kTmaWarps * kSlots * ITEM_BYTES;
+    static constexpr int SMEM = 1024 + RING_BYTES + kTmaWarps * kSlots * 8;
+};
+
+// Division of 32-bit unsigned integers by an invariant divisor d >= 1 with one
+// multiply-high, an add and two shifts, exact for every n < 2^32 (Granlund and
+// Montgomery, "Division by Invariant Integers using Multiplication", figure 4.1).
+struct FastDiv {
+    uint32_t mul, s1, s2;
+};
+
+FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while ((uint64_t(1) << l) < d) ++l;                 // ceil(log2 d)
+    FastDiv f;
+    f.mul = (uint32_t)((((uint64_t(1) << l) - d) << 32) / d + 1);
+    f.s1 = l < 1 ? l : 1;
+    f.s2 = l > 1 ? l - 1 : 0;
+    return f;
+}
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
+    const uint32_t t = __umulhi(n, f.mul);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+
+struct TmaParams {
+    uint32_t total_units;   // rows * K / E  (< 2^31)
+    uint32_t n_items;
+    uint32_t upr;           // units per row
+    FastDiv upr_div;
+};
+
+// Unit of the item read by lane pair `pair` in sub-step `sub`.  With 128-value units a
+// pair reads two flat rows; with 64-value units the order 0,2,4,6 | 1,3,5,7 | 8,10,..
+// keeps the four pairs of a quarter-warp on distinct swizzle phases.
+template <int E>
+__device__ __forceinline__ int item_unit(int pair, int sub) {
+    if constexpr (E == 128) return pair;
+    return sub * 16 + ((pair & 8) | ((pair & 3) << 1) | ((pair >> 2) & 1));
+}
+
+template <int G, int MODE>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    tma_unit_kernel(const __grid_constant__ CUtensorMap tmX, const UnitParams p,
+                    const TmaParams t, int* status) {
+    using S = TmaShape<G>;
+    constexpr int E = S::E;
+    constexpr int NCT = UnitShape<G>::NCT;
+    constexpr int SUBS = S::SUBS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING_BYTES);
+    __shared__ float red[32];
+    __shared__ float s_gsf;
+    __shared__ float inv_tab[128];
+    __shared__ int s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = lane & 1;
+    if (threadIdx.x == 0) s_abort = 0;
+    if (lane == 0)
+        for (int s = 0; s < kSlots; ++s) mbar_init(&full[warp * kSlots + s], 1);
+    fence_barrier_init();
+    __syncthreads();
+
+    float gsf = 0.0f;
+    if constexpr (MODE == 1) {
+        gsf = encode_prologue<kTmaThreads>(p, red, &s_gsf, inv_tab);
+        // scale bytes of the padding rows (up to the next multiple of 128) are zero
+        const int64_t pad_rows = (p.rows + 127) / 128 * 128 - p.rows;
+        for (int64_t i = (int64_t)blockIdx.x * kTmaThreads + threadIdx.x; i < pad_rows * p.cgroups;
+             i += (int64_t)gridDim.x * kTmaThreads) {
+            const int64_t row = p.rows + i / p.cgroups, cg = i % p.cgroups;
+            const int64_t off = (((row >> 7) * p.cgroups + cg) << 9) + ((row & 31) << 4) +
+                                (((row >> 5) & 3) << 2);
+            *reinterpret_cast<uint32_t*>(p.sf + off) = 0u;
+        }
+    }
+
+    const uint64_t policy = MODE == 0 ? l2_policy_evict_last() : l2_policy_evict_first();
+    const uint32_t stride = gridDim.x * kTmaWarps;
+    uint8_t* ring = smem + warp * kSlots * S::ITEM_BYTES;
+    uint64_t* bars = full + warp * kSlots;
+    const uint32_t first = blockIdx.x * kTmaWarps + warp;
+    if (lane == 0) {
+        for (int s = 0; s < kSlots; ++s) {
+            const uint32_t it = first + s * stride;
+            if (it < t.n_items) {
+                mbar_arrive_expect_tx(&bars[s], S::ITEM_BYTES);
+                tma_load_2d_hint(ring + s * S::ITEM_BYTES, &tmX, &bars[s], 0,
+                                 (int32_t)(it * kItemRows), policy);
+            }
+        }
+    }
+
+    const int pair = lane >> 1;
+    uint32_t tmax = 0u;
+    uint32_t k = 0;
+    for (uint32_t item = first; item < t.n_items; item += stride, ++k) {
+        const int s = (int)(k % kSlots);
+        if (!mbar_wait_bounded(&bars[s], (k / kSlots) & 1u, &s_abort, status, kTmaWaitBudgetNs))
+            break;
+        const uint8_t* slot = ring + s * S::ITEM_BYTES;
+        uint4 w[SUBS][NCT];
+#pragma unroll
+        for (int sub = 0; sub < SUBS; ++sub) {
+            const int m = item_unit<E>(pair, sub);
 #pragma unroll
             for (int i = 0; i < NCT; ++i) {
-                const float tm = absmax_words4(w[i]);
-                bm[i] = fmaxf(tm, __shfl_xor_sync(kFull, tm, 1));
+                const int j = 2 * i + h;                            // chunk of the unit
+                const int fr = (E == 128) ? 2 * m + (j >> 3) : m;   // flat row of the item
+                const int pos = (j & 7) ^ (fr & 7);
+                w[sub][i] = *reinterpret_cast<const uint4*>(slot + fr * 128 + pos * 16);
             }
-            uint32_t s8[NCT];
-#pragma unroll
-            for (int j = 0; j < NCT / 2; ++j) {
-                const float mine_bm = h ? bm[2 * j + 1] : bm[2 * j];
-                const uint32_t mine = e4m3_from_f32(__fdiv_rn(__fmul_rn(gsf, mine_bm), 6.0f));
-                const uint32_t other = __shfl_xor_sync(kFull, mine, 1);
-                s8[2 * j] = h ? other : mine;
-                s8[2 * j + 1] = h ? mine : other;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            const uint32_t nxt = item + kSlots * stride;
+            if (nxt < t.n_items) {
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&bars[s], S::ITEM_BYTES);
+                tma_load_2d_hint(ring + s * S::ITEM_BYTES, &tmX, &bars[s], 0,
+                                 (int32_t)(nxt * kItemRows), policy);
             }
-            uint32_t codes[NCT];
+        }
 #pragma unroll
-            for (int i = 0; i < NCT; ++i) {
-                // inv_tab[s8] = rn(gsf / dec(s8)); a zero scale zeroes the whole block
-                const float inv = inv_tab[s8[i]];
-                const float2 iv = make_float2(inv, inv);
-                const float2 a = mul2(word_to_f2(w[i].x), iv), b = mul2(word_to_f2(w[i].y), iv);
-                const float2 c = mul2(word_to_f2(w[i].z), iv), d = mul2(word_to_f2(w[i].w), iv);
-                const float q[8] = {a.x, a.y, b.x, b.y, c.x, c.y, d.x, d.y};
-                codes[i] = s8[i] ? e2m1x8_from_f32(q) : 0u;
-            }
-            // scale words: blocks 4q..4q+3 -> one aligned 32-bit word, lane h = q & 1
+        for (int sub = 0; sub < SUBS; ++sub) {
+            const uint32_t unit = item * S::UPI + item_unit<E>(pair, sub);
+            const bool active = unit < t.total_units;
+            const uint32_t row = fast_div(unit, t.upr_div);
+            const int64_t e0 = (int64_t)(unit - row * t.upr) * E;
+            if constexpr (G > 0) rotate_unit<G>(w[sub], h, p.hscale);
+            if constexpr (MODE == 0) {
 #pragma unroll
-            for (int q = 0; q < NCT / 4; ++q) {
-                if (active && (q & 1) == h) {
-                    const uint32_t word = s8[4 * q] | (s8[4 * q + 1] << 8) | (s8[4 * q + 2] << 16) |
-                                          (s8[4 * q + 3] << 24);
-                    const int64_t cg = e0 / 64 + q;
-                    const int64_t off = (((row >> 7) * p.cgroups + cg) << 9) + ((row & 31) << 4) +
-                                        (((row >> 5) & 3) << 2);
-                    *reinterpret_cast<uint32_t*>(p.sf + off) = word;
-                }
-            }
-            // packed bytes: each lane of the pair writes 16 contiguous bytes per 8-word half
-            const int valid_words = valid / 8;
-            uint8_t* dst = p.packed + row * (p.K / 2) + e0 / 2;
-            const bool al16 = ((row * (p.K / 2)) & 15) == 0;
-#pragma unroll
-            for (int hh = 0; hh < NCT / 4; ++hh) {
-                const uint32_t c0 = codes[4 * hh], c1 = codes[4 * hh + 1];
-                const uint32_t c2 = codes[4 * hh + 2], c3 = codes[4 * hh + 3];
-                const uint32_t r0 = __shfl_xor_sync(kFull, h ? c0 : c2, 1);
-                const uint32_t r1 = __shfl_xor_sync(kFull, h ? c1 : c3, 1);
-                const uint4 out = h ? make_uint4(r0, c2, r1, c3) : make_uint4(c0, r0, c1, r1);
-                const int wb = 8 * hh + 4 * h;
-                uint32_t* d = reinterpret_cast<uint32_t*>(dst + wb * 4);
-                if (data_row) {
-                    if (wb + 4 <= valid_words) {
-                        if (al16) {
-                            *reinterpret_cast<uint4*>(d) = out;
-                        } else {
-                            reinterpret_cast<uint2*>(d)[0] = make_uint2(out.x, out.y);
-                            reinterpret_cast<uint2*>(d)[1] = make_uint2(out.z, out.w);
-                        }
-                    } else {
-                        const uint32_t o[4] = {out.x, out.y, out.z, out.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            if (wb + j < valid_words) d[j] = o[j];
-                    }
-                }
+                for (int i = 0; i < NCT; ++i) tmax = absmax2_bf16(tmax, absmax_word4(w[sub][i]));
+            } else {
+                encode_unit<G>(w[sub], h, gsf, inv_tab, p, (int64_t)row, e0, E, active, active);
             }
         }
     }
     if constexpr (MODE == 0) {
-        const float m = block_max(tmax, red);
-        if (threadIdx.x == 0) p.partials_out[blockIdx.x] = m;
+        const float mx = block_max(absmax_of_pair(tmax), red);
+        if (threadIdx.x == 0) p.partials_out[blockIdx.x] = mx;
+    }
+    // after a timeout, let this warp's loads still in flight land before the CTA exits
+    if (s_abort && lane == 0) {
+        volatile int no_abort = 0;
+        for (uint32_t s = 0; s < (uint32_t)kSlots; ++s) {
+            const uint32_t kk = k + s;
+            const uint64_t it = first + (uint64_t)kk * stride;
+            if (it < t.n_items)
+                mbar_wait_bounded(&bars[kk % kSlots], (kk / kSlots) & 1u, &no_abort, nullptr,
+                                  100000000ull);
+        }
     }
 }
 
@@ -338,6 +549,50 @@ nvfp4_status dispatch(int g, const UnitParams& p, int grid, cudaStream_t stream)
         default: break;
     }
     return NVFP4_ERR_INVALID_ARG;
+}
+
+template <int G, int MODE>
+nvfp4_status launch_tma_unit(const CUtensorMap& map, const UnitParams& p, const TmaParams& t,
+                             int grid, int device, int* status, cudaStream_t stream) {
+    constexpr int smem = TmaShape<G>::SMEM;
+    static bool attr_set[64] = {false};
+    if (device < 0 || device >= 64) return NVFP4_ERR_DEVICE;
+    if (!attr_set[device]) {
+        if (cudaFuncSetAttribute(tma_unit_kernel<G, MODE>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        attr_set[device] = true;
+    }
+    tma_unit_kernel<G, MODE><<<grid, kTmaThreads, smem, stream>>>(map, p, t, status);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+template <int MODE>
+nvfp4_status dispatch_tma(int g, const CUtensorMap& map, const UnitParams& p, const TmaParams& t,
+                          int grid, int device, int* status, cudaStream_t stream) {
+    switch (g) {
+        case 0: return launch_tma_unit<0, MODE>(map, p, t, grid, device, status, stream);
+        case 16: return launch_tma_unit<16, MODE>(map, p, t, grid, device, status, stream);
+        case 32: return launch_tma_unit<32, MODE>(map, p, t, grid, device, status, stream);
+        case 64: return launch_tma_unit<64, MODE>(map, p, t, grid, device, status, stream);
+        case 128: return launch_tma_unit<128, MODE>(map, p, t, grid, device, status, stream);
+        default: break;
+    }
+    return NVFP4_ERR_INVALID_ARG;
+}
+
+// x as [rows*K/64, 64] bf16 with a [BR, 64] box and the 128-byte swizzle.
+bool make_flat_map(CUtensorMap* map, const void* x, int64_t flat_rows, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {64, (cuuint64_t)flat_rows};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(x), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 int64_t unit_elems(int g) { return g == 128 ? 128 : 64; }
@@ -373,6 +628,32 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
     p.gsf_out = gsf_out;
     p.gsf_w = gsf_w;
     p.alpha_out = alpha_out;
+
+    const int64_t flat_rows = rows * K / 64;
+    if (K % 64 == 0 && flat_rows < (int64_t(1) << 31) - 256) {
+        int* status = nullptr;
+        if ((st = status_word(&status)) != NVFP4_OK) return st;
+        CUtensorMap map;
+        if (!make_flat_map(&map, x, flat_rows, kItemRows)) return NVFP4_ERR_CUDA;
+        const int upi = group == 128 ? 16 : 32;
+        p.total_units = rows * p.upr;
+        TmaParams t;
+        t.total_units = (uint32_t)p.total_units;
+        t.n_items = (uint32_t)((p.total_units + upi - 1) / upi);
+        t.upr = (uint32_t)p.upr;
+        t.upr_div = make_fastdiv(t.upr);
+        const int64_t need = (t.n_items + kTmaWarps - 1) / kTmaWarps;
+        const int grid = (int)(need < dev.sms ? (need > 0 ? need : 1) : dev.sms);
+        if (gsf_in == nullptr) {
+            UnitParams a = p;
+            a.partials_out = partials;
+            st = dispatch_tma<0>(group, map, a, t, grid, dev.device, status, stream);
+            if (st != NVFP4_OK) return st;
+            p.partials = partials;
+            p.n_partials = grid;
+        }
+        return dispatch_tma<1>(group, map, p, t, grid, dev.device, status, stream);
+    }
 
     if (gsf_in == nullptr) {
         UnitParams a = p;

@@ -115,15 +115,18 @@ def test_hadamard_rotate(oracle, group, R, K):
 
 
 def test_format_conversions_exhaustive(oracle):
-    """The quantizer's device fp32 -> E2M1 and fp32 -> E4M3 conversions against the
-    oracle's encoders on all 2^32 fp32 bit patterns (NaNs excluded)."""
+    """The quantizer's device fp32 -> E2M1 and fp32 -> E4M3 conversions, and its
+    block-scale step E4M3(rn(y / 6)), against the oracle's encoders (the quotient
+    rounded by IEEE fp32 division) on all 2^32 fp32 bit patterns (NaNs excluded)."""
     n = 1 << 26
     e2 = torch.empty(n, dtype=torch.uint8, device=DEV)
     e4 = torch.empty(n, dtype=torch.uint8, device=DEV)
+    sc = torch.empty(n, dtype=torch.uint8, device=DEV)
     L = nv.lib()
     for chunk in range(1 << 6):
         first = chunk * n
-        assert L.nvfp4_debug_cvt_sweep(first, n, nv._ptr(e2), nv._ptr(e4), nv._stream()) == nv.OK
+        assert L.nvfp4_debug_cvt_sweep(first, n, nv._ptr(e2), nv._ptr(e4), nv._ptr(sc),
+                                       nv._stream()) == nv.OK
         v = (np.arange(n, dtype=np.uint32) + np.uint32(first)).view(np.float32)
         keep = ~np.isnan(v)
         vk = v[keep]
@@ -135,3 +138,7 @@ def test_format_conversions_exhaustive(oracle):
             o4 = oracle.e4m3_encode_array(vk)
             bad4 = np.flatnonzero(g4 != o4)
             assert bad4.size == 0, f"E4M3 differs for {vk[bad4[:6]]}: {g4[bad4[:6]]} vs {o4[bad4[:6]]}"
+            os_ = oracle.e4m3_encode_array(vk / np.float32(6.0))
+            gs = to_np(sc)[keep]
+            bads = np.flatnonzero(gs != os_)
+            assert bads.size == 0, f"scale differs for {vk[bads[:6]]}: {gs[bads[:6]]} vs {os_[bads[:6]]}"
