@@ -47,10 +47,10 @@ METRIC = "nvfp4_linear TFLOPS (% of dense FP4 peak); quantizer GB/s (% of HBM)"
 # null once the source has changed.  The quantizer figure is the qkv launch pair scaled
 # by the step's value count (traffic grows in proportion to the values).
 MEASURED_TRAFFIC = {
-    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "88cf5ad9245bf369",
-             "bytes_per_step": 545.6e6},
-    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "0099cc90a1a01db0",
-              "bytes_per_step": 138.1e6 * (3 * 32768 * 1024 + 32768 * 4096) / (32768 * 1024)},
+    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "27f2f54285285d48",
+             "bytes_per_step": 550.6e6},
+    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "687a039a27e3c813",
+              "bytes_per_step": 138.28e6 * (3 * 32768 * 1024 + 32768 * 4096) / (32768 * 1024)},
 }
 
 

@@ -23,7 +23,7 @@
  *  [P5] FastH3-QAD-v2 and NVFP4 VAE Decoders -- "The whole stack in NVFP4"
  *       (4-bit values plus one FP8 scale for every 16).
  *
- * Readings taken where the pages are silent (each also listed in the design doc):
+ * Readings taken where the pages are silent:
  *  R1 FP4_E4M3_RANGE = 448 * 6 = 2688 (largest E4M3 scale times largest E2M1 value).
  *  R2 dynamic global scale = 2688 / max(amax, 1e-12), amax over the whole call.
  *  R3 per-block order: bmax -> s_raw = rn(rn(gsf*bmax)/6) -> s8 = E4M3(s_raw) ->
