@@ -87,6 +87,9 @@ def lib():
         L.ora_hadamard_rotate.argtypes = [u16p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, u16p]
         L.ora_dequantize.restype = None
         L.ora_dequantize.argtypes = [u8p, u8p, ctypes.c_int64, ctypes.c_int64, f64p]
+        L.ora_dequantize_bf16.restype = None
+        L.ora_dequantize_bf16.argtypes = [u8p, u8p, ctypes.c_int64, ctypes.c_int64, ctypes.c_float,
+                                          u16p]
         L.ora_gemm_f64.restype = None
         L.ora_gemm_f64.argtypes = [u8p, u8p, u8p, u8p, ctypes.c_int64, ctypes.c_int64,
                                    ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
@@ -238,6 +241,15 @@ def dequantize(packed: np.ndarray, sf: np.ndarray, rows: int, K: int) -> np.ndar
     out = np.empty((rows, K), dtype=np.float64)
     lib().ora_dequantize(np.ascontiguousarray(packed).reshape(-1), np.ascontiguousarray(sf).reshape(-1),
                          rows, K, out.reshape(-1))
+    return out
+
+
+def dequantize_bf16(packed: np.ndarray, sf: np.ndarray, rows: int, K: int, gsf: float) -> np.ndarray:
+    """bf16 bits [rows, K] = RNE_bf16(fp32(E2M1(code) * E4M3(scale)) / gsf)."""
+    out = np.empty((rows, K), dtype=np.uint16)
+    lib().ora_dequantize_bf16(np.ascontiguousarray(packed).reshape(-1),
+                              np.ascontiguousarray(sf).reshape(-1), rows, K, np.float32(gsf),
+                              out.reshape(-1))
     return out
 
 

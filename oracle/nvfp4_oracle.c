@@ -305,6 +305,22 @@ EXPORT void ora_dequantize(const uint8_t* packed, const uint8_t* sf, int64_t R, 
         for (int64_t k = 0; k < K; ++k) out[r * K + k] = dequant_elem(packed, sf, r, k, K);
 }
 
+/* NVFP4 -> bf16 expansion of a packed tensor (the W4A16 path: "decode dynamic-scale
+ * NVFP4 H3 VAE tiles one at a time" -- FASTVIDEO_H3_ENCODER_FUSED_DEQUANT, which expands
+ * the serialized NVFP4 text encoder to bf16 on GPUs without an FP4 GEMM).  Reading: the
+ * value is E2M1(code) * E4M3(scale) (exact in fp32), divided by the global scale in fp32
+ * (IEEE, round to nearest even) and rounded to nearest even to bf16. */
+EXPORT void ora_dequantize_bf16(const uint8_t* packed, const uint8_t* sf, int64_t R, int64_t K,
+                                float gsf, uint16_t* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            const float v = (float)dequant_elem(packed, sf, r, k, K);
+            const float q = v / gsf;
+            out[r * K + k] = ora_f32_to_bf16(q);
+        }
+}
+
 /* y[i, n] = alpha * sum_k deq_a(rows[i], k) * deq_b(n, k) + bias[n], in fp64,
  * k ascending; every product is exact in fp64.  rows == NULL means rows 0..M-1
  * (then n_rows = M).  bias_bf16 may be NULL. */
