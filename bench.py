@@ -49,7 +49,7 @@ METRIC = "nvfp4_linear TFLOPS (% of dense FP4 peak); quantizer GB/s (% of HBM)"
 MEASURED_TRAFFIC = {
     "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "27f2f54285285d48",
              "bytes_per_step": 550.6e6},
-    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "687a039a27e3c813",
+    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "d22b82c548fc2926",
               "bytes_per_step": 138.28e6 * (3 * 32768 * 1024 + 32768 * 4096) / (32768 * 1024)},
 }
 
@@ -300,6 +300,32 @@ def weight_pack_rate(layers_src, dev):
             "bytes_per_value": 8.5625}
 
 
+def dequant_rate(dev):
+    """NVFP4 -> bf16 expansion of one 5120 x 25600 projection (131 M values; 74 MB in,
+    262 MB out, above L2), GB/s over the algorithmic 0.5 + 1/16 + 2 = 2.5625 B/value.  The
+    packed weight is an N(0, 0.02) weight quantized by nvfp4_quantize (untimed)."""
+    rows, K = 5120, 25600
+    w = W.qwen3_weight((rows, K), dev, W._gen(1005, dev))
+    packed, sf, gsf = nv.nvfp4_quantize(w, 0, None)
+    del w
+    y = torch.empty(rows, K, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        nv.nvfp4_dequantize(packed, sf, gsf, K, out=y)
+    torch.cuda.synchronize()
+    reps = 10
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        nv.nvfp4_dequantize(packed, sf, gsf, K, out=y)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    n = rows * K
+    gbps = n * 2.5625 / (ms * 1e-3) / 1e9
+    return {"values": n, "ms": ms, "GBps": gbps, "bytes_per_value": 2.5625,
+            "frac_of_measured_hbm": gbps / peaks()["hbm"]}
+
+
 def oracle_pack(layers_src):
     """The oracle's own weight packing (rotate g=128, dynamic quantize); untimed."""
     import oracle as O
@@ -359,12 +385,13 @@ def run_ours(args, dist_on, rank, world, local_rank):
     clk = None if args.kernels_only else clocks.stop()
     if args.kernels_only:        # profiling runs: the dynamic-scale step only
         s_total, s_q, s_g = total_ms, q_ms, g_ms
-        e2e_ms, h2d, d2h, wpack = float("nan"), 0, 0, None
+        e2e_ms, h2d, d2h, wpack, deq = float("nan"), 0, 0, None, None
     else:
         s_total, s_q, s_g = timed_steps(layers, False, args.steps, args.warmup, dist_on)
         e2e_ms, h2d, d2h = e2e_steps(layers, max(2, args.steps // 4), max(3, args.warmup),
                                      dist_on)
         wpack = weight_pack_rate(src, dev)
+        deq = dequant_rate(dev)
     assert nv.last_device_status() == nv.OK
 
     ms = max_over_ranks(total_ms / args.steps, dist_on)
@@ -405,6 +432,7 @@ def run_ours(args, dist_on, rank, world, local_rank):
         "static_scale": {"ms_per_step": s_ms, "TFLOP/s": aggregate_tflops(flops, s_ms, world),
                          "quantizer_ms": s_q, "gemm_ms": s_g},
         "weight_pack": wpack,
+        "dequant": deq,
         "e2e": {"value": aggregate_tflops(flops, e2e_ms, world), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "nvfp4_linear"},

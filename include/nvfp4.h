@@ -178,6 +178,24 @@ NVFP4_API nvfp4_status nvfp4_linear(const void* x_bf16, int64_t M, int64_t K, co
                           const void* bias_bf16, const float* gsf_x, int rotate_group,
                           void* workspace, size_t ws_bytes, void* y_bf16, void* stream);
 
+/*
+ * nvfp4_dequantize -- NVFP4 -> bf16 expansion of a packed tensor, the W4A16 path for
+ * GPUs without an FP4 GEMM ("decode dynamic-scale NVFP4 H3 VAE tiles one at a time" --
+ * FASTVIDEO_H3_ENCODER_FUSED_DEQUANT: one fused pass that expands the serialized NVFP4
+ * text encoder to bf16).
+ *   packed : in,  uint8 [rows, K/2] (element 2i in the low nibble of byte i)
+ *   sf     : in,  uint8 [nvfp4_scale_bytes(rows, K)], 128x4 layout
+ *   gsf    : in,  device fp32 scalar, the tensor's global scale
+ *   y_bf16 : out, bf16 [rows, K]
+ * y = RNE_bf16(fp32(E2M1(code) * E4M3(scale)) / gsf), the division in IEEE fp32.  Scale
+ * bytes are expected in 0..0x7E (what nvfp4_quantize writes); other bytes give the
+ * negative or NaN values their E4M3 decoding implies.  K % 16 == 0.
+ * Errors: INVALID_ARG, SHAPE (K <= 0 or K % 16), ALIGN (packed, sf, y not 16-byte
+ * aligned; gsf not 4-byte aligned), DEVICE, CUDA.
+ */
+NVFP4_API nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* sf, const float* gsf,
+                                        int64_t rows, int64_t K, void* y_bf16, void* stream);
+
 /* Size of the library's own fixed device scratch used by
  * nvfp4_linear_fixed_scratch: 8 MiB. */
 #define NVFP4_FIXED_SCRATCH_BYTES ((size_t)8 << 20)

@@ -35,6 +35,7 @@ SIGNATURES = {
     "nvfp4_quantize": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                               _vp]),
     "nvfp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "nvfp4_dequantize": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
     "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64]),
     "nvfp4_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _int, _vp, _sz, _vp,
                             _vp]),
@@ -190,6 +191,17 @@ def nvfp4_linear(x: torch.Tensor, w_packed: torch.Tensor, w_sf: torch.Tensor,
     _check("nvfp4_linear", lib().nvfp4_linear(
         _ptr(x), M, K, _ptr(w_packed), _ptr(w_sf), _ptr(gsf_w), N, _ptr(bias), _ptr(gsf_x),
         int(rotate_group), _ptr(workspace), workspace.numel(), _ptr(y), _stream(stream)))
+    return y
+
+
+def nvfp4_dequantize(packed: torch.Tensor, sf: torch.Tensor, gsf: torch.Tensor, K: int,
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """NVFP4 -> bf16: packed uint8 [rows, K/2] + 128x4 scales + device gsf -> bf16 [rows, K]."""
+    rows = packed.shape[0]
+    gsf = _scalar(gsf, packed.device, "gsf")
+    y = torch.empty(rows, K, dtype=torch.bfloat16, device=packed.device) if out is None else out
+    _check("nvfp4_dequantize", lib().nvfp4_dequantize(_ptr(packed), _ptr(sf), _ptr(gsf), rows, K,
+                                                      _ptr(y), _stream(stream)))
     return y
 
 

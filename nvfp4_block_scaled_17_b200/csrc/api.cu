@@ -206,6 +206,19 @@ nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
     return launch_gemm(a, sfa, b, sfb, alpha, bias, y, M, N, K, static_cast<cudaStream_t>(stream));
 }
 
+nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* sf, const float* gsf,
+                              int64_t rows, int64_t K, void* y, void* stream) {
+    if (!packed || !sf || !gsf || !y || rows < 0) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 16) return NVFP4_ERR_SHAPE;
+    if (!aligned(packed, 16) || !aligned(sf, 16) || !aligned(y, 16) || !aligned(gsf, 4))
+        return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (rows == 0) return NVFP4_OK;
+    return launch_dequantize(packed, sf, gsf, rows, K, y, static_cast<cudaStream_t>(stream));
+}
+
 size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K) {
     if (M < 0 || K <= 0) return 0;
     return linear_ws(M, K).total;

@@ -56,6 +56,13 @@ __device__ __forceinline__ float f32_from_e4m3(uint32_t b) {
     return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu)));
 }
 
+// fp32 value of an E2M1 code (bit 3 = sign; magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6).
+__device__ __forceinline__ float e2m1_value(uint32_t code) {
+    const uint32_t mag = code & 7u, e = mag >> 1, m = mag & 1u;
+    const float v = e ? (1.0f + 0.5f * (float)m) * (float)(1u << (e - 1)) : 0.5f * (float)m;
+    return (code & 8u) ? -v : v;
+}
+
 // Eight fp32 values -> eight E2M1 codes (RNE, saturating), element 0 in bits 0..3.
 __device__ __forceinline__ uint32_t e2m1x8_from_f32(const float (&v)[8]) {
     uint32_t out;
@@ -115,6 +122,28 @@ __device__ __forceinline__ float absmax_of_pair(uint32_t m) {
 
 __device__ __forceinline__ float absmax_words4(const uint4& w) {
     return absmax_of_pair(absmax_word4(w));
+}
+
+// Division of 32-bit unsigned integers by an invariant divisor d >= 1 with one
+// multiply-high, an add and two shifts, exact for every n < 2^32 (Granlund and
+// Montgomery, "Division by Invariant Integers using Multiplication", figure 4.1).
+struct FastDiv {
+    uint32_t mul, s1, s2;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while ((uint64_t(1) << l) < d) ++l;                 // ceil(log2 d)
+    FastDiv f;
+    f.mul = (uint32_t)((((uint64_t(1) << l) - d) << 32) / d + 1);
+    f.s1 = l < 1 ? l : 1;
+    f.s2 = l > 1 ? l - 1 : 0;
+    return f;
+}
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
+    const uint32_t t = __umulhi(n, f.mul);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
 }
 
 // ---------------------------------------------------------------------------

@@ -35,6 +35,10 @@ nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          const uint8_t* sfb, const float* alpha, const void* bias, void* y,
                          int64_t M, int64_t N, int64_t K, cudaStream_t stream);
 
+// NVFP4 -> bf16 expansion: y = bf16(fp32(E2M1 * E4M3) / gsf).
+nvfp4_status launch_dequantize(const uint8_t* packed, const uint8_t* sf, const float* gsf,
+                               int64_t rows, int64_t K, void* y, cudaStream_t stream);
+
 nvfp4_status launch_cvt_sweep(uint32_t first, int64_t n, uint8_t* e2m1, uint8_t* e4m3,
                               uint8_t* scale, cudaStream_t stream);
 nvfp4_status launch_wait_timeout(int64_t budget_us, cudaStream_t stream);

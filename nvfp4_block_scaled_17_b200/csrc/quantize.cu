@@ -377,28 +377,6 @@ struct TmaShape {
     static constexpr int SMEM = 1024 + RING_BYTES + kTmaWarps * kSlots * 8;
 };
 
-// Division of 32-bit unsigned integers by an invariant divisor d >= 1 with one
-// multiply-high, an add and two shifts, exact for every n < 2^32 (Granlund and
-// Montgomery, "Division by Invariant Integers using Multiplication", figure 4.1).
-struct FastDiv {
-    uint32_t mul, s1, s2;
-};
-
-FastDiv make_fastdiv(uint32_t d) {
-    uint32_t l = 0;
-    while ((uint64_t(1) << l) < d) ++l;                 // ceil(log2 d)
-    FastDiv f;
-    f.mul = (uint32_t)((((uint64_t(1) << l) - d) << 32) / d + 1);
-    f.s1 = l < 1 ? l : 1;
-    f.s2 = l > 1 ? l - 1 : 0;
-    return f;
-}
-
-__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
-    const uint32_t t = __umulhi(n, f.mul);
-    return (t + ((n - t) >> f.s1)) >> f.s2;
-}
-
 struct TmaParams {
     uint32_t total_units;   // rows * K / E  (< 2^31)
     uint32_t n_items;

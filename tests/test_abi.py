@@ -82,6 +82,11 @@ def test_gemm_and_linear_argument_errors(L):
     assert lin(A, 4, 96, A, A, A, 8, None, None, 0, A, 1 << 20, A, S) == nv.ERR_SHAPE
     assert lin(A, 4, 128, A, A, A, 8, None, None, 48, A, 1 << 20, A, S) == nv.ERR_INVALID_ARG
     assert lin(A, 4, 128, A, A, None, 8, None, None, 0, A, 1 << 20, A, S) == nv.ERR_INVALID_ARG
+    dq = L.nvfp4_dequantize
+    assert dq(None, A, A, 4, 64, A, S) == nv.ERR_INVALID_ARG
+    assert dq(A, A, A, 4, 24, A, S) == nv.ERR_SHAPE
+    assert dq(A, A, A, -1, 64, A, S) == nv.ERR_INVALID_ARG
+    assert dq(A, A, A, 4, 64, MIS, S) == nv.ERR_ALIGN
     fx = L.nvfp4_linear_fixed_scratch
     assert fx(A, 16384, 1024, A, A, A, 8, None, None, 0, A, S) == nv.ERR_WORKSPACE  # > 8 MiB
     assert fx(A, 4, 96, A, A, A, 8, None, None, 0, A, S) == nv.ERR_SHAPE
