@@ -152,6 +152,30 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const ui
                         const uint8_t* sfb, const float* alpha, const void* bias_bf16,
                         void* y_bf16, int64_t M, int64_t N, int64_t K, void* stream);
 
+/*
+ * nvfp4_gemm_quantize_out -- nvfp4_gemm whose epilogue hands the next linear its NVFP4
+ * input directly: the bf16 product y = bf16(alpha * acc + bias) is encoded in
+ * registers under a static global scale and only the codes and scales are written
+ * ("minimax_h3_nvfp4_decoder" -- NVFP4FusedState and NVFP4DecoderLinear.fused_state:
+ * the fused kernels quantize with a precomputed global scale and alpha, so dynamic
+ * scales and the activation rotation stay on the unfused path; "FastH3-QAD-v2 and NVFP4
+ * VAE Decoders" -- "Fused FP4 kernels": quantize, scale and GEMM without round trips
+ * through memory, bit-exact with the unfused path).
+ *   a, sfa, b, sfb, alpha, bias_bf16, M, N, K : as nvfp4_gemm
+ *   gsf_out    : in,  device fp32 scalar, the static global scale of the next linear's input
+ *   out_packed : out, uint8 [M, N/2]
+ *   out_sf     : out, uint8 [nvfp4_scale_bytes(M, N)], 128x4 layout, padding rows 0
+ * The encoding is exactly nvfp4_quantize(y, rotate_group 0, gsf_in = gsf_out) applied to
+ * the bf16 y nvfp4_gemm would have written; y itself is not written.  N % 64 == 0.
+ * Errors: as nvfp4_gemm; SHAPE also for N % 64; ALIGN for out_packed, out_sf (16 bytes)
+ * and gsf_out (4 bytes).
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_quantize_out(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                               const uint8_t* sfb, const float* alpha,
+                                               const void* bias_bf16, const float* gsf_out,
+                                               uint8_t* out_packed, uint8_t* out_sf, int64_t M,
+                                               int64_t N, int64_t K, void* stream);
+
 /* Workspace bytes nvfp4_linear needs for an [M, K] activation: the packed
  * activation, its scales, the two scalars and the dynamic-scale scratch, each
  * 256-byte aligned. */

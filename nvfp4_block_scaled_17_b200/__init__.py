@@ -36,6 +36,8 @@ SIGNATURES = {
                               _vp]),
     "nvfp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "nvfp4_dequantize": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
+    "nvfp4_gemm_quantize_out": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                       _i64, _vp]),
     "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64]),
     "nvfp4_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _int, _vp, _sz, _vp,
                             _vp]),
@@ -192,6 +194,25 @@ def nvfp4_linear(x: torch.Tensor, w_packed: torch.Tensor, w_sf: torch.Tensor,
         _ptr(x), M, K, _ptr(w_packed), _ptr(w_sf), _ptr(gsf_w), N, _ptr(bias), _ptr(gsf_x),
         int(rotate_group), _ptr(workspace), workspace.numel(), _ptr(y), _stream(stream)))
     return y
+
+
+def nvfp4_gemm_quantize_out(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,
+                            sfb: torch.Tensor, alpha: torch.Tensor, M: int, N: int, K: int,
+                            gsf_out: torch.Tensor, bias: torch.Tensor | None = None,
+                            out: tuple | None = None, stream=None):
+    """GEMM with the next linear's NVFP4 input as output: (packed uint8 [M, N/2], 128x4
+    scales) of bf16(alpha * A B^T + bias) under the static global scale gsf_out."""
+    alpha = _scalar(alpha, a.device, "alpha")
+    gsf_out = _scalar(gsf_out, a.device, "gsf_out")
+    if out is None:
+        packed = torch.empty(M, N // 2, dtype=torch.uint8, device=a.device)
+        sf = torch.empty(max(nvfp4_scale_bytes(M, N), 1), dtype=torch.uint8, device=a.device)
+    else:
+        packed, sf = out
+    _check("nvfp4_gemm_quantize_out", lib().nvfp4_gemm_quantize_out(
+        _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(alpha), _ptr(bias), _ptr(gsf_out),
+        _ptr(packed), _ptr(sf), M, N, K, _stream(stream)))
+    return packed, sf
 
 
 def nvfp4_dequantize(packed: torch.Tensor, sf: torch.Tensor, gsf: torch.Tensor, K: int,

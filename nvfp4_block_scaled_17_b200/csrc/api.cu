@@ -219,6 +219,27 @@ nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* sf, const fl
     return launch_dequantize(packed, sf, gsf, rows, K, y, static_cast<cudaStream_t>(stream));
 }
 
+nvfp4_status nvfp4_gemm_quantize_out(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                     const uint8_t* sfb, const float* alpha, const void* bias,
+                                     const float* gsf_out, uint8_t* out_packed, uint8_t* out_sf,
+                                     int64_t M, int64_t N, int64_t K, void* stream) {
+    if (!a || !sfa || !b || !sfb || !alpha || !gsf_out || !out_packed || !out_sf || M < 0 ||
+        N < 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 64 || K >= (int64_t(1) << 31) || N % 64) return NVFP4_ERR_SHAPE;
+    if (!aligned(a, 16) || !aligned(sfa, 16) || !aligned(b, 16) || !aligned(sfb, 16) ||
+        !aligned(out_packed, 16) || !aligned(out_sf, 16) || !aligned(alpha, 4) ||
+        !aligned(gsf_out, 4) || (bias && !aligned(bias, 16)))
+        return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    return launch_gemm_quant_out(a, sfa, b, sfb, alpha, bias, gsf_out, out_packed, out_sf, M, N,
+                                 K, static_cast<cudaStream_t>(stream));
+}
+
 size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K) {
     if (M < 0 || K <= 0) return 0;
     return linear_ws(M, K).total;

@@ -77,11 +77,42 @@ struct GemmParams {
     int sf_row_tiles_b;        // ceil(N / 128)
     int tma_store;             // 1: y through the tensor map (N % 8 == 0)
     int n_fast;                // tile order: 1 = consecutive tiles walk N (B re-read from L2)
+    // quantized output (the NVFP4 input of the next linear), when the kernel is built for it
+    uint8_t* q_packed;         // [M, N/2]
+    uint8_t* q_sf;             // 128x4 scales of an [M, N] operand
+    const float* q_gsf;        // static global scale of the next linear's input
+    int q_cgroups;             // N / 64
     int* status;
     uint64_t budget_ns;
 };
 
 __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) { return bf16x2_rn(lo, hi); }
+
+// NVFP4 encoding of one 16-value block given as 8 bf16 pairs, exactly as the activation
+// quantizer encodes it under a static global scale: bmax, E4M3 scale of rn(gsf*bmax)/6,
+// codes E2M1(rn(x * rn(gsf / scale))), all codes 0 under a zero scale.  Returns the
+// scale byte; c0 / c1 receive the codes of values 0..7 / 8..15.
+template <int OFF>
+__device__ __forceinline__ uint32_t quantize_block(const uint32_t (&words)[16], float gsf,
+                                                   uint32_t& c0, uint32_t& c1) {
+    const uint32_t* w = words + OFF;   // compile-time offset: the array stays in registers
+    const uint32_t tm = absmax2_bf16(absmax2_bf16(absmax2_bf16(w[0], w[1]), absmax2_bf16(w[2], w[3])),
+                                     absmax2_bf16(absmax2_bf16(w[4], w[5]), absmax2_bf16(w[6], w[7])));
+    const uint32_t s8 = e4m3_scale_of_scaled_max(__fmul_rn(gsf, absmax_of_pair(tm)));
+    const float inv = (s8 == 0u || s8 == 127u) ? 0.0f : __fdiv_rn(gsf, f32_from_e4m3(s8));
+    float q[2][8];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t x = w[4 * h + j];
+            q[h][2 * j] = __fmul_rn(__uint_as_float(x << 16), inv);
+            q[h][2 * j + 1] = __fmul_rn(__uint_as_float(x & 0xffff0000u), inv);
+        }
+    c0 = s8 ? e2m1x8_from_f32(q[0]) : 0u;
+    c1 = s8 ? e2m1x8_from_f32(q[1]) : 0u;
+    return s8;
+}
 
 // Tile order.  The CTAs of one wave work on consecutive tiles; walking N first keeps
 // the few A row blocks of a wave hot while the (smaller) B panel is re-read from L2,
@@ -96,6 +127,7 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& 
     }
 }
 
+template <bool QOUT>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
@@ -250,6 +282,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const int quad = warp & 3;
         const int half = (warp - 2) >> 2;
         const float alpha = *p.alpha;
+        const float qgsf = QOUT ? *p.q_gsf : 0.0f;
         uint8_t* stg = sStg + (warp - 2) * 2 * STG_BYTES;
         int stg_sel = 0;
         int it = 0;
@@ -269,10 +302,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             const bool owns_overlap = (b == 0) ? (half == 1) : (half == 0);
             const uint32_t buf_col = b ? TMEM_BUF1 : 0u;
             const int row0 = m_blk * BM + quad * 32;
-            // bf16(alpha * acc + bias) of one 32-column chunk, staged and stored
-            auto store_chunk = [&](const uint32_t (&r)[32], int chunk) {
-                const int n0 = n_blk * BN + chunk * 32;
-                if (n0 >= p.N) return;   // warp-uniform
+            // bf16(alpha * acc + bias) of one 32-column chunk, as 16 bf16 pairs
+            auto make_words = [&](const uint32_t (&r)[32], int n0, uint32_t (&packed)[16]) {
                 float bv[32];
                 if (p.bias) {
                     if (n0 + 32 <= p.N) {
@@ -291,7 +322,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                             bv[j] = __uint_as_float((uint32_t)p.bias[min(n0 + j, p.N - 1)] << 16);
                     }
                 }
-                uint32_t packed[16];
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
                     float v0 = __fmul_rn(alpha, __uint_as_float(r[j]));
@@ -302,6 +332,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     }
                     packed[j / 2] = bf16x2_bits(v0, v1);
                 }
+            };
+            // the bf16 chunk, staged and stored
+            auto store_words = [&](const uint32_t (&packed)[16], int n0) {
                 if (p.tma_store) {
                     uint8_t* sb = stg + stg_sel * STG_BYTES;
                     if (lane == 0) bulk_wait_read<1>();   // this buffer's previous store
@@ -350,8 +383,35 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acc_free[b]);
                 }
-                store_chunk(r0, c0);
-                store_chunk(r1, c1);
+                const int n00 = n_blk * BN + c0 * 32, n01 = n_blk * BN + c1 * 32;
+                uint32_t w0[16], w1[16];
+                if (n00 < p.N) make_words(r0, n00, w0);   // warp-uniform
+                if (n01 < p.N) make_words(r1, n01, w1);
+                if constexpr (!QOUT) {
+                    if (n00 < p.N) store_words(w0, n00);
+                    if (n01 < p.N) store_words(w1, n01);
+                }
+                if constexpr (QOUT) {
+                    // chunks c0, c1 are the 64 columns of one 4-block scale word (N % 64 == 0)
+                    if (n00 < p.N) {
+                        const int row = row0 + lane;
+                        uint32_t codes[8];
+                        const uint32_t s0 = quantize_block<0>(w0, qgsf, codes[0], codes[1]);
+                        const uint32_t s1 = quantize_block<8>(w0, qgsf, codes[2], codes[3]);
+                        const uint32_t s2 = quantize_block<0>(w1, qgsf, codes[4], codes[5]);
+                        const uint32_t s3 = quantize_block<8>(w1, qgsf, codes[6], codes[7]);
+                        const bool live = row < p.M;       // padding rows get zero scales
+                        const uint32_t word = live ? (s0 | (s1 << 8) | (s2 << 16) | (s3 << 24)) : 0u;
+                        const size_t off = ((size_t)(row >> 7) * p.q_cgroups + (size_t)(n00 >> 6)) * 512 +
+                                           (size_t)((row & 31) << 4) + (size_t)(((row >> 5) & 3) << 2);
+                        *reinterpret_cast<uint32_t*>(p.q_sf + off) = word;
+                        if (live) {
+                            uint4* dst = reinterpret_cast<uint4*>(p.q_packed + (size_t)row * (p.N / 2) + n00 / 2);
+                            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                        }
+                    }
+                }
             }
         }
         if (lane == 0) bulk_wait_all();
@@ -397,9 +457,21 @@ bool make_output_map(CUtensorMap* map, void* base, int64_t M, int64_t N) {
 
 }  // namespace
 
-nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
-                         const uint8_t* sfb, const float* alpha, const void* bias, void* y,
-                         int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+namespace {
+
+// Quantized-output request of the fused epilogue (the next linear's NVFP4 input; the
+// bf16 product itself is not written).
+struct QuantOut {
+    uint8_t* packed;
+    uint8_t* sf;
+    const float* gsf;
+};
+
+template <bool QOUT>
+nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                              const uint8_t* sfb, const float* alpha, const void* bias, void* y,
+                              int64_t M, int64_t N, int64_t K, const QuantOut* q,
+                              cudaStream_t stream) {
     DeviceInfo dev;
     nvfp4_status st = device_info(&dev);
     if (st != NVFP4_OK) return st;
@@ -409,7 +481,7 @@ nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
     CUtensorMap mapA, mapB, mapY;
     if (!make_operand_map(&mapA, a, M, K / 2, BM) || !make_operand_map(&mapB, b, N, K / 2, BN))
         return NVFP4_ERR_CUDA;
-    const bool tma_store = (N % 8) == 0;
+    const bool tma_store = !QOUT && (N % 8) == 0;
     if (tma_store) {
         if (!make_output_map(&mapY, y, M, N)) return NVFP4_ERR_CUDA;
     } else {
@@ -418,7 +490,7 @@ nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
 
     static bool attr_set[64] = {false};
     if (!attr_set[dev.device & 63]) {
-        if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemm_kernel<QOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  SMEM_BYTES) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         attr_set[dev.device & 63] = true;
@@ -439,13 +511,35 @@ nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
     p.sf_row_tiles_b = (int)((N + 127) / 128);
     p.tma_store = tma_store ? 1 : 0;
     p.n_fast = (N <= M) ? 1 : 0;
+    if (QOUT) {
+        p.q_packed = q->packed;
+        p.q_sf = q->sf;
+        p.q_gsf = q->gsf;
+        p.q_cgroups = (int)(N / 64);
+    }
     p.status = status;
     p.budget_ns = 4000000000ull;   // 4 s
 
     const int tiles = p.m_blocks * p.n_blocks;
     const int grid = tiles < dev.sms ? tiles : dev.sms;
-    gemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(mapA, mapB, mapY, p);
+    gemm_kernel<QOUT><<<grid, THREADS, SMEM_BYTES, stream>>>(mapA, mapB, mapY, p);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+}  // namespace
+
+nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                         const uint8_t* sfb, const float* alpha, const void* bias, void* y,
+                         int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    return launch_gemm_impl<false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, nullptr, stream);
+}
+
+nvfp4_status launch_gemm_quant_out(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                   const uint8_t* sfb, const float* alpha, const void* bias,
+                                   const float* gsf_out, uint8_t* out_packed, uint8_t* out_sf,
+                                   int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    QuantOut q{out_packed, out_sf, gsf_out};
+    return launch_gemm_impl<true>(a, sfa, b, sfb, alpha, bias, nullptr, M, N, K, &q, stream);
 }
 
 }  // namespace nvfp4

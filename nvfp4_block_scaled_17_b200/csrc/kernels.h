@@ -35,6 +35,13 @@ nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          const uint8_t* sfb, const float* alpha, const void* bias, void* y,
                          int64_t M, int64_t N, int64_t K, cudaStream_t stream);
 
+// The GEMM whose epilogue emits the NVFP4 encoding of its bf16 output instead of the
+// output itself (static global scale gsf_out, 128x4 scales, N % 64 == 0).
+nvfp4_status launch_gemm_quant_out(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                   const uint8_t* sfb, const float* alpha, const void* bias,
+                                   const float* gsf_out, uint8_t* out_packed, uint8_t* out_sf,
+                                   int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+
 // NVFP4 -> bf16 expansion: y = bf16(fp32(E2M1 * E4M3) / gsf).
 nvfp4_status launch_dequantize(const uint8_t* packed, const uint8_t* sf, const float* gsf,
                                int64_t rows, int64_t K, void* y, cudaStream_t stream);

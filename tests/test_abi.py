@@ -82,6 +82,10 @@ def test_gemm_and_linear_argument_errors(L):
     assert lin(A, 4, 96, A, A, A, 8, None, None, 0, A, 1 << 20, A, S) == nv.ERR_SHAPE
     assert lin(A, 4, 128, A, A, A, 8, None, None, 48, A, 1 << 20, A, S) == nv.ERR_INVALID_ARG
     assert lin(A, 4, 128, A, A, None, 8, None, None, 0, A, 1 << 20, A, S) == nv.ERR_INVALID_ARG
+    gq = L.nvfp4_gemm_quantize_out
+    assert gq(A, A, A, A, A, None, A, A, A, 4, 96, 64, S) == nv.ERR_SHAPE      # N % 64
+    assert gq(A, A, A, A, A, None, None, A, A, 4, 64, 64, S) == nv.ERR_INVALID_ARG
+    assert gq(A, A, A, A, A, None, A, MIS, A, 4, 64, 64, S) == nv.ERR_ALIGN
     dq = L.nvfp4_dequantize
     assert dq(None, A, A, 4, 64, A, S) == nv.ERR_INVALID_ARG
     assert dq(A, A, A, 4, 24, A, S) == nv.ERR_SHAPE
