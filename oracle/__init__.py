@@ -28,6 +28,7 @@ _lib = None
 u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
 u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
 f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
 i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
 
 
@@ -87,6 +88,13 @@ def lib():
         L.ora_hadamard_rotate.argtypes = [u16p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, u16p]
         L.ora_dequantize.restype = None
         L.ora_dequantize.argtypes = [u8p, u8p, ctypes.c_int64, ctypes.c_int64, f64p]
+        i8p = np.ctypeslib.ndpointer(dtype=np.int8, flags="C_CONTIGUOUS")
+        i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+        L.ora_int8_quantize_rows.restype = None
+        L.ora_int8_quantize_rows.argtypes = [u16p, ctypes.c_int64, ctypes.c_int64, i8p, f32p]
+        L.ora_int8_gemm_f64.restype = None
+        L.ora_int8_gemm_f64.argtypes = [i8p, f32p, i8p, f32p, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, f64p]
         L.ora_dequantize_bf16.restype = None
         L.ora_dequantize_bf16.argtypes = [u8p, u8p, ctypes.c_int64, ctypes.c_int64, ctypes.c_float,
                                           u16p]
@@ -94,7 +102,6 @@ def lib():
         L.ora_gemm_f64.argtypes = [u8p, u8p, u8p, u8p, ctypes.c_int64, ctypes.c_int64,
                                    ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_int64, f64p]
-        f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
         for name in ("ora_e2m1_encode_array", "ora_e4m3_encode_array"):
             getattr(L, name).restype = None
             getattr(L, name).argtypes = [f32p, ctypes.c_int64, u8p]
@@ -251,6 +258,32 @@ def dequantize_bf16(packed: np.ndarray, sf: np.ndarray, rows: int, K: int, gsf: 
                               np.ascontiguousarray(sf).reshape(-1), rows, K, np.float32(gsf),
                               out.reshape(-1))
     return out
+
+
+def int8_quantize_rows(x: np.ndarray):
+    """bf16 [R, K] -> (int8 codes [R, K], fp32 row scales [R]) (per-row amax / 127)."""
+    x = _u16(x)
+    R, K = x.shape
+    q = np.empty((R, K), dtype=np.int8)
+    s = np.empty(R, dtype=np.float32)
+    lib().ora_int8_quantize_rows(x.reshape(-1), R, K, q.reshape(-1), s)
+    return q, s
+
+
+def int8_gemm_f64(qx: np.ndarray, sx: np.ndarray, qw: np.ndarray, sw: np.ndarray,
+                  bias: np.ndarray | None = None, rows: np.ndarray | None = None) -> np.ndarray:
+    """fp64 y[rows, N] = s_x[m] s_w[n] sum_k qx qw + bias."""
+    M, K = qx.shape
+    N = qw.shape[0]
+    rows_arr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    n_rows = M if rows_arr is None else rows_arr.size
+    y = np.empty((n_rows, N), dtype=np.float64)
+    bias_arr = None if bias is None else np.ascontiguousarray(_u16(bias).reshape(-1))
+    lib().ora_int8_gemm_f64(np.ascontiguousarray(qx).reshape(-1), np.ascontiguousarray(sx, dtype=np.float32),
+                            np.ascontiguousarray(qw).reshape(-1), np.ascontiguousarray(sw, dtype=np.float32),
+                            N, K, None if bias_arr is None else bias_arr.ctypes.data,
+                            None if rows_arr is None else rows_arr.ctypes.data, n_rows, y.reshape(-1))
+    return y
 
 
 def gemm_f64(a: np.ndarray, sfa: np.ndarray, b: np.ndarray, sfb: np.ndarray, M: int, N: int,

@@ -364,3 +364,59 @@ EXPORT float ora_quantize(const uint16_t* x, int64_t R, int64_t K, float gsf_in,
     ora_scale_swizzle(sf_lin_scratch, R, K, sf);
     return gsf;
 }
+
+/* ------------------------------------------------------------------------- */
+/* int8 per-row W8A8 linear ("FastH3-4-step-Preview-v1-r16-int8", "What is    */
+/* inside": weight = round(W / scale) clamped to -127..127 with scale =       */
+/* amax(|W[row]|) / 127 per output row; activations quantized per row at call */
+/* time and multiplied with an int8 GEMM).                                     */
+/* Readings: the division and the scale are fp32 (IEEE, round to nearest      */
+/* even); round() is half to even; an all-zero row has scale 0 and codes 0;   */
+/* activations use the same per-row rule; the product is                      */
+/* y = bf16(fp32(fp32(acc) * s_x[m]) * s_w[n] + bias[n]) with an exact integer */
+/* accumulator.                                                                */
+/* ------------------------------------------------------------------------- */
+
+/* Row r of x (bf16 [R, K]) -> int8 codes and the fp32 row scale. */
+EXPORT void ora_int8_quantize_rows(const uint16_t* x, int64_t R, int64_t K, int8_t* q,
+                                   float* scale) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(ora_bf16_to_f32(x[r * K + k]));
+            if (a > amax) amax = a;
+        }
+        const float s = amax / 127.0f;
+        scale[r] = s;
+        for (int64_t k = 0; k < K; ++k) {
+            int8_t c = 0;
+            if (s != 0.0f) {
+                const float v = ora_bf16_to_f32(x[r * K + k]) / s;
+                double t = nearbyint((double)v);          /* half to even (default mode) */
+                if (t > 127.0) t = 127.0;
+                if (t < -127.0) t = -127.0;
+                c = (int8_t)t;
+            }
+            q[r * K + k] = c;
+        }
+    }
+}
+
+/* y[i, n] = s_x[m] * s_w[n] * sum_k qx[m, k] qw[n, k] + bias[n] in fp64 (the integer sum
+ * exact), rows as in ora_gemm_f64. */
+EXPORT void ora_int8_gemm_f64(const int8_t* qx, const float* sx, const int8_t* qw,
+                              const float* sw, int64_t N, int64_t K, const uint16_t* bias_bf16,
+                              const int64_t* rows, int64_t n_rows, double* y) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < n_rows; ++i) {
+        int64_t m = rows ? rows[i] : i;
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t acc = 0;
+            for (int64_t k = 0; k < K; ++k) acc += (int64_t)qx[m * K + k] * (int64_t)qw[n * K + k];
+            double v = (double)acc * (double)sx[m] * (double)sw[n];
+            if (bias_bf16) v += (double)ora_bf16_to_f32(bias_bf16[n]);
+            y[i * N + n] = v;
+        }
+    }
+}
