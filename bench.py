@@ -358,6 +358,57 @@ def fused_chain(src, dev):
             "fused_gemm_TFLOPs": 2.0 * M * N1 * K1 / (t_g * 1e-3) / 1e12}
 
 
+def int8_block(src, dev, pk):
+    """The same four ViT-block linears (M = 32768) on the int8 per-row W8A8 path: per
+    linear, the per-row activation quantizer then the int8 GEMM (weights quantized
+    offline, untimed).  TOPS against the int8 dense peak (2 x the measured bf16 figure,
+    nominal ratio 4.5 / 2.25); the quantizer's GB/s over 2 B read + 1 B + 4 B / row written."""
+    layers = []
+    for l in src:
+        wq, sw = nv.int8_quantize_rows(l.weight)
+        M, K = l.x.shape
+        layers.append(dict(x=l.x, wq=wq, sw=sw, bias=l.bias, M=M, K=K, N=l.N,
+                           xq=torch.empty(M, K, dtype=torch.int8, device=dev),
+                           sx=torch.empty(M, dtype=torch.float32, device=dev),
+                           y=torch.empty(M, l.N, dtype=torch.bfloat16, device=dev)))
+
+    def step(evs=None):
+        for i, L_ in enumerate(layers):
+            if evs is not None:
+                evs[i][0].record()
+            nv.int8_quantize_rows(L_["x"], out=(L_["xq"], L_["sx"]))
+            if evs is not None:
+                evs[i][1].record()
+            nv.int8_gemm(L_["xq"], L_["sx"], L_["wq"], L_["sw"], L_["bias"], out=L_["y"])
+            if evs is not None:
+                evs[i][2].record()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    reps = 10
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in layers] for _ in range(reps)]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for k in range(reps):
+        step(evs[k])
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    q_ms = sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(reps) for i in range(4)) / reps
+    g_ms = sum(evs[k][i][1].elapsed_time(evs[k][i][2]) for k in range(reps) for i in range(4)) / reps
+    ops = sum(2.0 * L_["M"] * L_["N"] * L_["K"] for L_ in layers)
+    qbytes = sum(L_["M"] * L_["K"] * 3.0 + L_["M"] * 4.0 for L_ in layers)
+    i8_peak = 2.0 * pk["bf16_sus"]
+    g_tops = ops / (g_ms * 1e-3) / 1e12
+    return {"workload": "ViT block linears, M=32768, int8 per-row W8A8",
+            "ms_per_step": ms, "TOPS": ops / (ms * 1e-3) / 1e12,
+            "gemm_ms": g_ms, "gemm_TOPS": g_tops, "gemm_frac_of_int8_peak": g_tops / i8_peak,
+            "int8_peak_TOPS": i8_peak, "quantizer_ms": q_ms,
+            "quantizer_GBps": qbytes / (q_ms * 1e-3) / 1e9,
+            "quantizer_frac_of_hbm": qbytes / (q_ms * 1e-3) / 1e9 / pk["hbm"]}
+
+
 def dequant_rate(dev):
     """NVFP4 -> bf16 expansion of one 5120 x 25600 projection (131 M values; 74 MB in,
     262 MB out, above L2), GB/s over the algorithmic 0.5 + 1/16 + 2 = 2.5625 B/value.  The
@@ -443,7 +494,7 @@ def run_ours(args, dist_on, rank, world, local_rank):
     clk = None if args.kernels_only else clocks.stop()
     if args.kernels_only:        # profiling runs: the dynamic-scale step only
         s_total, s_q, s_g = total_ms, q_ms, g_ms
-        e2e_ms, h2d, d2h, wpack, deq, fchain = float("nan"), 0, 0, None, None, None
+        e2e_ms, h2d, d2h, wpack, deq, fchain, i8 = float("nan"), 0, 0, None, None, None, None
     else:
         s_total, s_q, s_g = timed_steps(layers, False, args.steps, args.warmup, dist_on)
         e2e_ms, h2d, d2h = e2e_steps(layers, max(2, args.steps // 4), max(3, args.warmup),
@@ -451,6 +502,7 @@ def run_ours(args, dist_on, rank, world, local_rank):
         wpack = weight_pack_rate(src, dev)
         deq = dequant_rate(dev)
         fchain = fused_chain(src, dev)
+        i8 = int8_block(src, dev, pk)
     assert nv.last_device_status() == nv.OK
 
     ms = max_over_ranks(total_ms / args.steps, dist_on)
@@ -493,6 +545,7 @@ def run_ours(args, dist_on, rank, world, local_rank):
         "weight_pack": wpack,
         "dequant": deq,
         "fused_chain": fchain,
+        "int8_linear": i8,
         "e2e": {"value": aggregate_tflops(flops, e2e_ms, world), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "nvfp4_linear"},

@@ -220,6 +220,53 @@ NVFP4_API nvfp4_status nvfp4_linear(const void* x_bf16, int64_t M, int64_t K, co
 NVFP4_API nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* sf, const float* gsf,
                                         int64_t rows, int64_t K, void* y_bf16, void* stream);
 
+/* ---- int8 per-row W8A8 linear ------------------------------------------------ */
+/*
+ * The pages' second quantized linear ("FastH3-4-step-Preview-v1-r16-int8" -- "What is
+ * inside"): int8 codes round(x / s) clamped to -127..127 with one fp32 scale
+ * s = amax(|row|) / 127 per row, weights per output row offline and activations per row
+ * at call time; the product runs on the int8 tensor cores with an exact int32
+ * accumulator.  Division and scale in fp32 (round to nearest even), round() half to
+ * even, an all-zero row gives s = 0 and codes 0.
+ */
+
+/*
+ * int8_quantize_rows -- per-row int8 quantizer.
+ *   x_bf16 : in,  bf16 [rows, K], K % 16 == 0
+ *   q      : out, int8 [rows, K]
+ *   scale  : out, fp32 [rows]
+ * Errors: INVALID_ARG, SHAPE (K <= 0 or K % 16), ALIGN (x, q 16-byte; scale 4-byte),
+ * DEVICE, CUDA.
+ */
+NVFP4_API nvfp4_status int8_quantize_rows(const void* x_bf16, int64_t rows, int64_t K, int8_t* q,
+                                          float* scale, void* stream);
+
+/*
+ * int8_gemm -- y = bf16((fp32(acc) * sa[m]) * sb[n] + bias[n]), acc = sum_k a[m,k] b[n,k]
+ * in int32 (tcgen05.mma kind::i8).
+ *   a, sa : in, int8 [M, K] and fp32 [M];  b, sb : in, int8 [N, K] and fp32 [N]
+ *   bias_bf16 : in, bf16 [N] or NULL;  y_bf16 : out, bf16 [M, N]
+ * K % 32 == 0.  Errors: as nvfp4_gemm (ALIGN: a, b, y, bias 16-byte; sa, sb 16-byte).
+ */
+NVFP4_API nvfp4_status int8_gemm(const int8_t* a, const float* sa, const int8_t* b, const float* sb,
+                                 const void* bias_bf16, void* y_bf16, int64_t M, int64_t N,
+                                 int64_t K, void* stream);
+
+/* Workspace bytes int8_linear needs for an [M, K] activation: the codes and the row
+ * scales, 256-byte aligned. */
+NVFP4_API size_t int8_linear_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * int8_linear -- int8_quantize_rows(x) then int8_gemm with the stored weight, one stream.
+ *   x_bf16 : in, bf16 [M, K];  wq, sw : in, int8 [N, K] and fp32 [N] (offline codes)
+ *   bias_bf16 : in, bf16 [N] or NULL;  workspace : int8_linear_workspace_bytes(M, K) bytes,
+ *   256-byte aligned;  y_bf16 : out, bf16 [M, N].  K % 32 == 0.
+ * Errors: as int8_quantize_rows and int8_gemm; WORKSPACE.
+ */
+NVFP4_API nvfp4_status int8_linear(const void* x_bf16, int64_t M, int64_t K, const int8_t* wq,
+                                   const float* sw, int64_t N, const void* bias_bf16,
+                                   void* workspace, size_t ws_bytes, void* y_bf16, void* stream);
+
 /* Size of the library's own fixed device scratch used by
  * nvfp4_linear_fixed_scratch: 8 MiB. */
 #define NVFP4_FIXED_SCRATCH_BYTES ((size_t)8 << 20)

@@ -36,6 +36,10 @@ SIGNATURES = {
                               _vp]),
     "nvfp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
     "nvfp4_dequantize": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
+    "int8_quantize_rows": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "int8_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "int8_linear_workspace_bytes": (_sz, [_i64, _i64]),
+    "int8_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp, _vp]),
     "nvfp4_gemm_quantize_out": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
                                        _i64, _vp]),
     "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64]),
@@ -213,6 +217,54 @@ def nvfp4_gemm_quantize_out(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,
         _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(alpha), _ptr(bias), _ptr(gsf_out),
         _ptr(packed), _ptr(sf), M, N, K, _stream(stream)))
     return packed, sf
+
+
+# ---------------------------------------------------------------------------
+# int8 per-row W8A8 linear
+# ---------------------------------------------------------------------------
+
+def int8_quantize_rows(x: torch.Tensor, out: tuple | None = None, stream=None):
+    """bf16 [rows, K] -> (int8 codes [rows, K], fp32 row scales [rows])."""
+    _bf16_2d(x, "x")
+    R, K = x.shape
+    if out is None:
+        q = torch.empty(R, K, dtype=torch.int8, device=x.device)
+        s = torch.empty(max(R, 1), dtype=torch.float32, device=x.device)
+    else:
+        q, s = out
+    _check("int8_quantize_rows", lib().int8_quantize_rows(_ptr(x), R, K, _ptr(q), _ptr(s),
+                                                          _stream(stream)))
+    return q, s
+
+
+def int8_gemm(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb: torch.Tensor,
+              bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """y bf16 [M, N] = bf16((fp32(a b^T) * sa[m]) * sb[n] + bias)."""
+    M, K = a.shape
+    N = b.shape[0]
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=a.device) if out is None else out
+    _check("int8_gemm", lib().int8_gemm(_ptr(a), _ptr(sa), _ptr(b), _ptr(sb), _ptr(bias), _ptr(y),
+                                        M, N, K, _stream(stream)))
+    return y
+
+
+def int8_linear(x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                bias: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The int8 per-row linear: bf16 x [M, K] with stored int8 codes wq [N, K] and scales
+    sw [N] -> bf16 [M, N]."""
+    _bf16_2d(x, "x")
+    M, K = x.shape
+    N = wq.shape[0]
+    if workspace is None:
+        workspace = torch.empty(max(int(lib().int8_linear_workspace_bytes(M, K)), 1),
+                                dtype=torch.uint8, device=x.device)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check("int8_linear", lib().int8_linear(_ptr(x), M, K, _ptr(wq), _ptr(sw), N, _ptr(bias),
+                                            _ptr(workspace), workspace.numel(), _ptr(y),
+                                            _stream(stream)))
+    return y
 
 
 def nvfp4_dequantize(packed: torch.Tensor, sf: torch.Tensor, gsf: torch.Tensor, K: int,

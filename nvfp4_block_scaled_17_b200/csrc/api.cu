@@ -240,6 +240,63 @@ nvfp4_status nvfp4_gemm_quantize_out(const uint8_t* a, const uint8_t* sfa, const
                                  K, static_cast<cudaStream_t>(stream));
 }
 
+nvfp4_status int8_quantize_rows(const void* x, int64_t rows, int64_t K, int8_t* q, float* scale,
+                                void* stream) {
+    if (!x || !q || !scale || rows < 0) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 16) return NVFP4_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale, 4)) return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (rows == 0) return NVFP4_OK;
+    return launch_int8_quantize_rows(x, rows, K, q, scale, static_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status int8_gemm(const int8_t* a, const float* sa, const int8_t* b, const float* sb,
+                       const void* bias, void* y, int64_t M, int64_t N, int64_t K, void* stream) {
+    if (!a || !sa || !b || !sb || !y || M < 0 || N < 0) return NVFP4_ERR_INVALID_ARG;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 32 || K >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(y, 16) || !aligned(sa, 16) ||
+        !aligned(sb, 16) || (bias && !aligned(bias, 16)))
+        return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    return launch_int8_gemm(a, sa, b, sb, bias, y, M, N, K, static_cast<cudaStream_t>(stream));
+}
+
+size_t int8_linear_workspace_bytes(int64_t M, int64_t K) {
+    if (M < 0 || K <= 0) return 0;
+    return align256((size_t)M * (size_t)K) + align256((size_t)M * 4);
+}
+
+nvfp4_status int8_linear(const void* x, int64_t M, int64_t K, const int8_t* wq, const float* sw,
+                         int64_t N, const void* bias, void* workspace, size_t ws_bytes, void* y,
+                         void* stream) {
+    if (!x || !wq || !sw || !y || M < 0 || N < 0) return NVFP4_ERR_INVALID_ARG;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 32 || K >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(sw, 16) || !aligned(y, 16) ||
+        (bias && !aligned(bias, 16)))
+        return NVFP4_ERR_ALIGN;
+    const size_t need = int8_linear_workspace_bytes(M, K);
+    if (!workspace || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    int8_t* xq = static_cast<int8_t*>(workspace);
+    float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                         align256((size_t)M * (size_t)K));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_int8_quantize_rows(x, M, K, xq, sx, s);
+    if (st != NVFP4_OK) return st;
+    return launch_int8_gemm(xq, sx, wq, sw, bias, y, M, N, K, s);
+}
+
 size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K) {
     if (M < 0 || K <= 0) return 0;
     return linear_ws(M, K).total;

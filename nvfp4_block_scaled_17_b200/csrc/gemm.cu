@@ -63,6 +63,9 @@ constexpr int SF_SLOTS = 5;             // 12 columns each: 4 for A, 8 for B (25
 // N = 256, M = 128, dense K = 64.
 constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                            ((uint32_t)(BM >> 4) << 24);
+// kind::i8: int32 accumulator (D format 2), signed int8 A and B (format 1), K-major.
+constexpr uint32_t IDESC_I8 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                              ((uint32_t)(BM >> 4) << 24);
 
 struct GemmParams {
     const uint8_t* sfa;
@@ -82,6 +85,9 @@ struct GemmParams {
     uint8_t* q_sf;             // 128x4 scales of an [M, N] operand
     const float* q_gsf;        // static global scale of the next linear's input
     int q_cgroups;             // N / 64
+    // int8 operands (the W8A8 linear): fp32 row scales of A and of B
+    const float* sx;
+    const float* sw;
     int* status;
     uint64_t budget_ns;
 };
@@ -127,7 +133,7 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& 
     }
 }
 
-template <bool QOUT>
+template <bool QOUT, bool I8>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
@@ -192,17 +198,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                         break;
                     }
                     const int steps = min(4, p.kchunks - 4 * kt);
-                    const uint32_t sf_bytes = (uint32_t)steps * 512u;
+                    const uint32_t sf_bytes = I8 ? 0u : (uint32_t)steps * 512u;
                     mbar_arrive_expect_tx(&full[stage], SMEM_A + SMEM_B + sf_bytes * (1 + sfb_tiles));
                     tma_load_2d(sA + stage * SMEM_A, &tmA, &full[stage], kt * BKB, m_blk * BM);
                     tma_load_2d(sB + stage * SMEM_B, &tmB, &full[stage], kt * BKB, n_blk * BN);
-                    bulk_load(sSFA + stage * SMEM_SFA,
-                              p.sfa + ((size_t)m_blk * p.kchunks + 4 * kt) * 512, sf_bytes,
-                              &full[stage]);
-                    for (int t = 0; t < sfb_tiles; ++t)
-                        bulk_load(sSFB + stage * SMEM_SFB + t * 2048,
-                                  p.sfb + ((size_t)(2 * n_blk + t) * p.kchunks + 4 * kt) * 512,
-                                  sf_bytes, &full[stage]);
+                    if constexpr (!I8) {
+                        bulk_load(sSFA + stage * SMEM_SFA,
+                                  p.sfa + ((size_t)m_blk * p.kchunks + 4 * kt) * 512, sf_bytes,
+                                  &full[stage]);
+                        for (int t = 0; t < sfb_tiles; ++t)
+                            bulk_load(sSFB + stage * SMEM_SFB + t * 2048,
+                                      p.sfb + ((size_t)(2 * n_blk + t) * p.kchunks + 4 * kt) * 512,
+                                      sf_bytes, &full[stage]);
+                    }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -252,15 +260,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     const uint32_t sfa0 = smem_u32(sSFA + stage * SMEM_SFA);
                     const uint32_t sfb0 = smem_u32(sSFB + stage * SMEM_SFB);
                     for (int kk = 0; kk < steps; ++kk) {
-                        const uint32_t sfa_t = tmem + TMEM_SF + 12u * (uint32_t)sf_slot;
-                        const uint32_t sfb_t = sfa_t + 4;
-                        tc_copy_sf(sfa_t, sdesc_sf(sfa0 + 512 * kk));
-                        tc_copy_sf(sfb_t, sdesc_sf(sfb0 + 512 * kk));
-                        tc_copy_sf(sfb_t + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
-                        mma_nvf4(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
-                                 sdesc_kmajor_sw128(b0 + 32 * kk), IDESC, sfa_t, sfb_t,
-                                 (kt | kk) != 0);
-                        if (++sf_slot == SF_SLOTS) sf_slot = 0;
+                        if constexpr (I8) {
+                            mma_i8(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
+                                   sdesc_kmajor_sw128(b0 + 32 * kk), IDESC_I8, (kt | kk) != 0);
+                        } else {
+                            const uint32_t sfa_t = tmem + TMEM_SF + 12u * (uint32_t)sf_slot;
+                            const uint32_t sfb_t = sfa_t + 4;
+                            tc_copy_sf(sfa_t, sdesc_sf(sfa0 + 512 * kk));
+                            tc_copy_sf(sfb_t, sdesc_sf(sfb0 + 512 * kk));
+                            tc_copy_sf(sfb_t + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
+                            mma_nvf4(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
+                                     sdesc_kmajor_sw128(b0 + 32 * kk), IDESC, sfa_t, sfb_t,
+                                     (kt | kk) != 0);
+                            if (++sf_slot == SF_SLOTS) sf_slot = 0;
+                        }
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == STAGES) {
@@ -281,7 +294,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         // epilogue: quadrant q = warp % 4 (tensor-memory lanes 32q..32q+31), column half h
         const int quad = warp & 3;
         const int half = (warp - 2) >> 2;
-        const float alpha = *p.alpha;
+        const float alpha = I8 ? 0.0f : *p.alpha;
         const float qgsf = QOUT ? *p.q_gsf : 0.0f;
         uint8_t* stg = sStg + (warp - 2) * 2 * STG_BYTES;
         int stg_sel = 0;
@@ -302,33 +315,45 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             const bool owns_overlap = (b == 0) ? (half == 1) : (half == 0);
             const uint32_t buf_col = b ? TMEM_BUF1 : 0u;
             const int row0 = m_blk * BM + quad * 32;
+            const float sx_row = (I8 && row0 + lane < p.M) ? p.sx[row0 + lane] : 0.0f;
             // bf16(alpha * acc + bias) of one 32-column chunk, as 16 bf16 pairs
             auto make_words = [&](const uint32_t (&r)[32], int n0, uint32_t (&packed)[16]) {
-                float bv[32];
+                // the bias as 16 bf16 pairs, widened pair by pair below
+                uint32_t bw[16];
                 if (p.bias) {
                     if (n0 + 32 <= p.N) {
                         const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0);
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             const uint4 w = bp[q4];
-                            bv[8 * q4 + 0] = bf16lo(w.x); bv[8 * q4 + 1] = bf16hi(w.x);
-                            bv[8 * q4 + 2] = bf16lo(w.y); bv[8 * q4 + 3] = bf16hi(w.y);
-                            bv[8 * q4 + 4] = bf16lo(w.z); bv[8 * q4 + 5] = bf16hi(w.z);
-                            bv[8 * q4 + 6] = bf16lo(w.w); bv[8 * q4 + 7] = bf16hi(w.w);
+                            bw[4 * q4] = w.x; bw[4 * q4 + 1] = w.y;
+                            bw[4 * q4 + 2] = w.z; bw[4 * q4 + 3] = w.w;
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            bv[j] = __uint_as_float((uint32_t)p.bias[min(n0 + j, p.N - 1)] << 16);
+                        for (int j = 0; j < 16; ++j)
+                            bw[j] = (uint32_t)p.bias[min(n0 + 2 * j, p.N - 1)] |
+                                    ((uint32_t)p.bias[min(n0 + 2 * j + 1, p.N - 1)] << 16);
                     }
                 }
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
-                    float v0 = __fmul_rn(alpha, __uint_as_float(r[j]));
-                    float v1 = __fmul_rn(alpha, __uint_as_float(r[j + 1]));
+                    float v0, v1;
+                    if constexpr (I8) {
+                        // (fp32(acc) * s_x[row]) * s_w[col], s_w read per column pair
+                        const float2 sw2 = (n0 + j + 1 < p.N)
+                                               ? *reinterpret_cast<const float2*>(p.sw + n0 + j)
+                                               : make_float2(p.sw[min(n0 + j, p.N - 1)],
+                                                             p.sw[min(n0 + j + 1, p.N - 1)]);
+                        v0 = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sx_row), sw2.x);
+                        v1 = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 1]), sx_row), sw2.y);
+                    } else {
+                        v0 = __fmul_rn(alpha, __uint_as_float(r[j]));
+                        v1 = __fmul_rn(alpha, __uint_as_float(r[j + 1]));
+                    }
                     if (p.bias) {
-                        v0 = __fadd_rn(v0, bv[j]);
-                        v1 = __fadd_rn(v1, bv[j + 1]);
+                        v0 = __fadd_rn(v0, bf16lo(bw[j / 2]));
+                        v1 = __fadd_rn(v1, bf16hi(bw[j / 2]));
                     }
                     packed[j / 2] = bf16x2_bits(v0, v1);
                 }
@@ -467,19 +492,23 @@ struct QuantOut {
     const float* gsf;
 };
 
-template <bool QOUT>
+// One launcher for the three builds of the kernel: NVFP4 (sfa/sfb = 128x4 scales,
+// alpha), NVFP4 with the quantized output, and int8 (sfa/sfb unused; sx/sw = fp32 row
+// scales of A and B).
+template <bool QOUT, bool I8>
 nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                               const uint8_t* sfb, const float* alpha, const void* bias, void* y,
                               int64_t M, int64_t N, int64_t K, const QuantOut* q,
-                              cudaStream_t stream) {
+                              const float* sx, const float* sw, cudaStream_t stream) {
     DeviceInfo dev;
     nvfp4_status st = device_info(&dev);
     if (st != NVFP4_OK) return st;
     int* status = nullptr;
     if ((st = status_word(&status)) != NVFP4_OK) return st;
 
+    const int64_t kbytes = I8 ? K : K / 2;   // bytes of one operand row
     CUtensorMap mapA, mapB, mapY;
-    if (!make_operand_map(&mapA, a, M, K / 2, BM) || !make_operand_map(&mapB, b, N, K / 2, BN))
+    if (!make_operand_map(&mapA, a, M, kbytes, BM) || !make_operand_map(&mapB, b, N, kbytes, BN))
         return NVFP4_ERR_CUDA;
     const bool tma_store = !QOUT && (N % 8) == 0;
     if (tma_store) {
@@ -490,7 +519,7 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
 
     static bool attr_set[64] = {false};
     if (!attr_set[dev.device & 63]) {
-        if (cudaFuncSetAttribute(gemm_kernel<QOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gemm_kernel<QOUT, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  SMEM_BYTES) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         attr_set[dev.device & 63] = true;
@@ -506,8 +535,10 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
     p.N = (int)N;
     p.m_blocks = (int)((M + BM - 1) / BM);
     p.n_blocks = (int)((N + BN - 1) / BN);
-    p.k_tiles = (int)((K + 255) / 256);
-    p.kchunks = (int)(K / 64);
+    p.k_tiles = (int)((kbytes + BKB - 1) / BKB);
+    p.kchunks = (int)(kbytes / 32);          // 32-byte MMA K steps
+    p.sx = sx;
+    p.sw = sw;
     p.sf_row_tiles_b = (int)((N + 127) / 128);
     p.tma_store = tma_store ? 1 : 0;
     p.n_fast = (N <= M) ? 1 : 0;
@@ -522,7 +553,7 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
 
     const int tiles = p.m_blocks * p.n_blocks;
     const int grid = tiles < dev.sms ? tiles : dev.sms;
-    gemm_kernel<QOUT><<<grid, THREADS, SMEM_BYTES, stream>>>(mapA, mapB, mapY, p);
+    gemm_kernel<QOUT, I8><<<grid, THREADS, SMEM_BYTES, stream>>>(mapA, mapB, mapY, p);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
@@ -531,7 +562,8 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
 nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          const uint8_t* sfb, const float* alpha, const void* bias, void* y,
                          int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
-    return launch_gemm_impl<false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, nullptr, stream);
+    return launch_gemm_impl<false, false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, nullptr,
+                                          nullptr, nullptr, stream);
 }
 
 nvfp4_status launch_gemm_quant_out(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
@@ -539,7 +571,16 @@ nvfp4_status launch_gemm_quant_out(const uint8_t* a, const uint8_t* sfa, const u
                                    const float* gsf_out, uint8_t* out_packed, uint8_t* out_sf,
                                    int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
     QuantOut q{out_packed, out_sf, gsf_out};
-    return launch_gemm_impl<true>(a, sfa, b, sfb, alpha, bias, nullptr, M, N, K, &q, stream);
+    return launch_gemm_impl<true, false>(a, sfa, b, sfb, alpha, bias, nullptr, M, N, K, &q,
+                                         nullptr, nullptr, stream);
+}
+
+nvfp4_status launch_int8_gemm(const int8_t* a, const float* sa, const int8_t* b, const float* sb,
+                              const void* bias, void* y, int64_t M, int64_t N, int64_t K,
+                              cudaStream_t stream) {
+    return launch_gemm_impl<false, true>(reinterpret_cast<const uint8_t*>(a), nullptr,
+                                         reinterpret_cast<const uint8_t*>(b), nullptr, nullptr,
+                                         bias, y, M, N, K, nullptr, sa, sb, stream);
 }
 
 }  // namespace nvfp4

@@ -42,6 +42,13 @@ nvfp4_status launch_gemm_quant_out(const uint8_t* a, const uint8_t* sfa, const u
                                    const float* gsf_out, uint8_t* out_packed, uint8_t* out_sf,
                                    int64_t M, int64_t N, int64_t K, cudaStream_t stream);
 
+// int8 per-row W8A8: row quantizer and GEMM with y = bf16((acc * sa[m]) * sb[n] + bias).
+nvfp4_status launch_int8_quantize_rows(const void* x, int64_t rows, int64_t K, int8_t* q,
+                                       float* scale, cudaStream_t stream);
+nvfp4_status launch_int8_gemm(const int8_t* a, const float* sa, const int8_t* b, const float* sb,
+                              const void* bias, void* y, int64_t M, int64_t N, int64_t K,
+                              cudaStream_t stream);
+
 // NVFP4 -> bf16 expansion: y = bf16(fp32(E2M1 * E4M3) / gsf).
 nvfp4_status launch_dequantize(const uint8_t* packed, const uint8_t* sf, const float* gsf,
                                int64_t rows, int64_t K, void* y, cudaStream_t stream);
