@@ -41,16 +41,15 @@ from nvfp4_block_scaled_17_b200 import workloads as W  # noqa: E402
 
 METRIC = "nvfp4_linear TFLOPS (% of dense FP4 peak); quantizer GB/s (% of HBM)"
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one step, from the ncu
-# captures summarised in profiles/ (gemm_kernel_vit_block.md, unit_kernel_vit_qkv.md),
-# valid only for the kernel sources they were taken on (sha256 prefix); reported as
-# null once the source has changed.  The quantizer figure is the qkv launch pair scaled
-# by the step's value count (traffic grows in proportion to the values).
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one step's launches (4
+# GEMMs, 8 quantizer passes), from the ncu capture summarised in
+# profiles/vit_block_step_launches.md, valid only for the kernel sources it was taken on
+# (sha256 prefix); reported as null once a source has changed.
 MEASURED_TRAFFIC = {
-    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "27f2f54285285d48",
-             "bytes_per_step": 550.6e6},
-    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "d22b82c548fc2926",
-              "bytes_per_step": 138.28e6 * (3 * 32768 * 1024 + 32768 * 4096) / (32768 * 1024)},
+    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "eec3e6d02cf3a787",
+             "bytes_per_step": 530.4e6},
+    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "aec233f10454b338",
+              "bytes_per_step": 959.3e6},
 }
 
 

@@ -43,28 +43,37 @@ __global__ void __launch_bounds__(kI8Threads) int8_rows_kernel(const uint16_t* _
         const bool fast = s >= 1.17549435e-38f;
         const float r = fast ? __frcp_rn(s) : 0.0f;
         int8_t* qr = q + row * K;
-        for (int64_t k = 8 * lane; k < K; k += 256) {
-            const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t out[2] = {0u, 0u};
-            if (s != 0.0f) {
+        // one loop per case, so the inner loop carries no per-value branch
+        auto encode = [=](auto quotient) {
+            for (int64_t k = 8 * lane; k < K; k += 256) {
+                const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                int c[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint32_t word = w[j >> 1];
-                    const float xv = __uint_as_float((j & 1) ? (word & 0xffff0000u) : (word << 16));
-                    float qt;
-                    if (fast) {
-                        const float q0 = __fmul_rn(xv, r);
-                        qt = __fmaf_rn(__fmaf_rn(-q0, s, xv), r, q0);
-                    } else {
-                        qt = __fdiv_rn(xv, s);
-                    }
-                    int c = __float2int_rn(qt);
-                    c = c > 127 ? 127 : (c < -127 ? -127 : c);
-                    out[j >> 2] |= ((uint32_t)c & 0xffu) << (8 * (j & 3));
+                    c[j] = __float2int_rn(quotient(
+                        __uint_as_float((j & 1) ? (word & 0xffff0000u) : (word << 16))));
                 }
+                uint32_t out[2];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    out[hh] = __byte_perm(__byte_perm(c[4 * hh], c[4 * hh + 1], 0x0040),
+                                          __byte_perm(c[4 * hh + 2], c[4 * hh + 3], 0x0040), 0x5410);
+                *reinterpret_cast<uint2*>(qr + k) = make_uint2(out[0], out[1]);
             }
-            *reinterpret_cast<uint2*>(qr + k) = make_uint2(out[0], out[1]);
+        };
+        // |x| <= amax keeps |x / s| <= 127 (1 + 2^-23): the rounded code is within -127..127
+        // without a clamp.
+        if (fast) {
+            encode([r, s](float xv) {
+                const float q0 = __fmul_rn(xv, r);
+                return __fmaf_rn(__fmaf_rn(-q0, s, xv), r, q0);
+            });
+        } else if (s != 0.0f) {
+            encode([s](float xv) { return __fdiv_rn(xv, s); });
+        } else {
+            encode([](float) { return 0.0f; });
         }
     }
 }

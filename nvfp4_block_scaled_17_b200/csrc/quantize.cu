@@ -510,6 +510,203 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Single pass for a dynamic scale when the whole call fits in shared memory at once
+// (every warp's items fit its three ring slots; 14.5 M values on 148 SMs -- a 4096 x
+// 1024 tile is 4.2 M).  Each warp loads its items once, rotates them in place in shared
+// memory while taking the amax, the CTAs meet at a grid barrier (cooperative launch, so
+// all of them are resident; the wait is bounded), and every warp then encodes its items
+// from shared memory with the global scale: one HBM read and one rotation instead of two.
+// The arithmetic is the two-pass kernels' own, so the results are identical.
+// ---------------------------------------------------------------------------
+
+template <int G>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    single_pass_kernel(const __grid_constant__ CUtensorMap tmX, const UnitParams p,
+                       const TmaParams t, float* partials, unsigned int* arrive, int* status) {
+    using S = TmaShape<G>;
+    constexpr int E = S::E;
+    constexpr int NCT = UnitShape<G>::NCT;
+    constexpr int SUBS = S::SUBS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING_BYTES);
+    __shared__ float red[32];
+    __shared__ float s_gsf;
+    __shared__ float inv_tab[128];
+    __shared__ int s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = lane & 1;
+    const int pair = lane >> 1;
+    if (threadIdx.x == 0) s_abort = 0;
+    if (lane == 0)
+        for (int s = 0; s < kSlots; ++s) mbar_init(&full[warp * kSlots + s], 1);
+    fence_barrier_init();
+    __syncthreads();
+
+    const uint32_t stride = gridDim.x * kTmaWarps;
+    const uint32_t first = blockIdx.x * kTmaWarps + warp;
+    uint8_t* ring = smem + warp * kSlots * S::ITEM_BYTES;
+    uint64_t* bars = full + warp * kSlots;
+    if (lane == 0)
+        for (int k = 0; k < kSlots; ++k) {
+            const uint32_t it = first + k * stride;
+            if (it < t.n_items) {
+                mbar_arrive_expect_tx(&bars[k], S::ITEM_BYTES);
+                tma_load_2d(ring + k * S::ITEM_BYTES, &tmX, &bars[k], 0, (int32_t)(it * kItemRows));
+            }
+        }
+
+    // the swizzled position of chunk i of sub-unit `sub` of this lane in an item
+    auto chunk_ptr = [&](uint8_t* slot, int sub, int i) -> uint4* {
+        const int m = item_unit<E>(pair, sub);
+        const int j = 2 * i + h;
+        const int fr = (E == 128) ? 2 * m + (j >> 3) : m;
+        return reinterpret_cast<uint4*>(slot + fr * 128 + (((j & 7) ^ (fr & 7)) << 4));
+    };
+
+    // pass over the own items: rotate in place, amax of the rotated values
+    uint32_t tmax = 0u;
+    bool ok = true;
+    for (int k = 0; k < kSlots; ++k) {
+        const uint32_t item = first + k * stride;
+        if (item >= t.n_items) break;
+        if (!mbar_wait_bounded(&bars[k], 0u, &s_abort, status, kTmaWaitBudgetNs)) {
+            ok = false;
+            break;
+        }
+        uint8_t* slot = ring + k * S::ITEM_BYTES;
+#pragma unroll
+        for (int sub = 0; sub < SUBS; ++sub) {
+            uint4 w[NCT];
+#pragma unroll
+            for (int i = 0; i < NCT; ++i) w[i] = *chunk_ptr(slot, sub, i);
+            if constexpr (G > 0) {
+                rotate_unit<G>(w, h, p.hscale);
+#pragma unroll
+                for (int i = 0; i < NCT; ++i) *chunk_ptr(slot, sub, i) = w[i];
+            }
+            // units past the end hold the zeros the copy filled in: they add nothing
+#pragma unroll
+            for (int i = 0; i < NCT; ++i) tmax = absmax2_bf16(tmax, absmax_word4(w[i]));
+        }
+    }
+    if (!ok) {
+        // let this warp's other loads land before the CTA can leave
+        if (lane == 0) {
+            volatile int no_abort = 0;
+            for (int k = 0; k < kSlots; ++k)
+                if (first + k * stride < t.n_items)
+                    mbar_wait_bounded(&bars[k], 0u, &no_abort, nullptr, 100000000ull);
+        }
+    }
+
+    // grid-wide amax: per-CTA partials, then a bounded barrier on the arrival count
+    const float m = block_max(absmax_of_pair(tmax), red);
+    if (threadIdx.x == 0) {
+        partials[blockIdx.x] = m;
+        __threadfence();
+        atomicAdd(arrive, 1u);
+        const uint64_t t0 = globaltimer_ns();
+        while (atomicAdd(arrive, 0u) < gridDim.x) {
+            if (s_abort || globaltimer_ns() - t0 > kTmaWaitBudgetNs) {
+                record_status(status, NVFP4_ERR_TIMEOUT);
+                s_abort = 1;
+                break;
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    if (s_abort) return;
+
+    // the global scale from every CTA's partial (read past L1), then the encode table
+    float mm = 0.0f;
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += kTmaThreads) mm = fmaxf(mm, __ldcg(partials + i));
+    mm = block_max(mm, red);
+    if (threadIdx.x == 0) s_gsf = __fdiv_rn(kFp4E4m3Range, fmaxf(mm, kAmaxFloor));
+    __syncthreads();
+    const float gsf = s_gsf;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (p.gsf_out) *p.gsf_out = gsf;
+        if (p.alpha_out) *p.alpha_out = __fdiv_rn(1.0f, __fmul_rn(gsf, *p.gsf_w));
+    }
+    if (threadIdx.x < 128) {
+        const float sv = f32_from_e4m3(threadIdx.x);
+        inv_tab[threadIdx.x] = (threadIdx.x == 0 || threadIdx.x == 127) ? 0.0f : __fdiv_rn(gsf, sv);
+    }
+    // scale bytes of the padding rows (up to the next multiple of 128) are zero
+    const int64_t pad_rows = (p.rows + 127) / 128 * 128 - p.rows;
+    for (int64_t i = (int64_t)blockIdx.x * kTmaThreads + threadIdx.x; i < pad_rows * p.cgroups;
+         i += (int64_t)gridDim.x * kTmaThreads) {
+        const int64_t row = p.rows + i / p.cgroups, cg = i % p.cgroups;
+        const int64_t off = (((row >> 7) * p.cgroups + cg) << 9) + ((row & 31) << 4) +
+                            (((row >> 5) & 3) << 2);
+        *reinterpret_cast<uint32_t*>(p.sf + off) = 0u;
+    }
+    __syncthreads();
+
+    // encode the own items from shared memory
+    for (int k = 0; k < kSlots; ++k) {
+        const uint32_t item = first + k * stride;
+        if (item >= t.n_items) break;
+        uint8_t* slot = ring + k * S::ITEM_BYTES;
+#pragma unroll
+        for (int sub = 0; sub < SUBS; ++sub) {
+            uint4 w[NCT];
+#pragma unroll
+            for (int i = 0; i < NCT; ++i) w[i] = *chunk_ptr(slot, sub, i);
+            const uint32_t unit = item * S::UPI + item_unit<E>(pair, sub);
+            const bool active = unit < t.total_units;
+            const uint32_t row = fast_div(unit, t.upr_div);
+            const int64_t e0 = (int64_t)(unit - row * t.upr) * E;
+            encode_unit<G>(w, h, gsf, inv_tab, p, (int64_t)row, e0, E, active, active);
+        }
+    }
+}
+
+template <int G>
+nvfp4_status launch_single_pass(const CUtensorMap& map, const UnitParams& p, const TmaParams& t,
+                                int grid, float* partials, int device, int* status,
+                                cudaStream_t stream) {
+    constexpr int smem = TmaShape<G>::SMEM;
+    static bool attr_set[64] = {false};
+    if (device < 0 || device >= 64) return NVFP4_ERR_DEVICE;
+    if (!attr_set[device]) {
+        if (cudaFuncSetAttribute(single_pass_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        attr_set[device] = true;
+    }
+    // the arrival counter lives in the last word of the caller's 4 KiB workspace
+    unsigned int* arrive = reinterpret_cast<unsigned int*>(partials) + (kMaxPartials - 1);
+    if (cudaMemsetAsync(arrive, 0, sizeof(unsigned int), stream) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    const CUtensorMap* mp = &map;
+    void* args[] = {const_cast<CUtensorMap*>(mp), const_cast<UnitParams*>(&p),
+                    const_cast<TmaParams*>(&t), &partials, &arrive, &status};
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(single_pass_kernel<G>), dim3(grid),
+                                    dim3(kTmaThreads), args, smem, stream) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
+
+nvfp4_status dispatch_single_pass(int g, const CUtensorMap& map, const UnitParams& p,
+                                  const TmaParams& t, int grid, float* partials, int device,
+                                  int* status, cudaStream_t stream) {
+    switch (g) {
+        case 0: return launch_single_pass<0>(map, p, t, grid, partials, device, status, stream);
+        case 16: return launch_single_pass<16>(map, p, t, grid, partials, device, status, stream);
+        case 32: return launch_single_pass<32>(map, p, t, grid, partials, device, status, stream);
+        case 64: return launch_single_pass<64>(map, p, t, grid, partials, device, status, stream);
+        case 128: return launch_single_pass<128>(map, p, t, grid, partials, device, status, stream);
+        default: break;
+    }
+    return NVFP4_ERR_INVALID_ARG;
+}
+
 template <int G, int MODE>
 nvfp4_status launch_unit(const UnitParams& p, int grid, cudaStream_t stream) {
     unit_kernel<G, MODE><<<grid, kThreads, 0, stream>>>(p);
@@ -620,6 +817,14 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
         t.n_items = (uint32_t)((p.total_units + upi - 1) / upi);
         t.upr = (uint32_t)p.upr;
         t.upr_div = make_fastdiv(t.upr);
+        // dynamic scale that fits on chip: one pass, every warp holding at most kSlots items
+        const int64_t per_cta = (int64_t)kTmaWarps * kSlots;
+        if (gsf_in == nullptr && (int64_t)t.n_items <= (int64_t)dev.sms * per_cta) {
+            // as many CTAs as give every warp one item, up to one per SM
+            const int64_t g1 = ((int64_t)t.n_items + kTmaWarps - 1) / kTmaWarps;
+            return dispatch_single_pass(group, map, p, t, (int)(g1 < dev.sms ? (g1 > 0 ? g1 : 1) : dev.sms),
+                                        partials, dev.device, status, stream);
+        }
         const int64_t need = (t.n_items + kTmaWarps - 1) / kTmaWarps;
         const int grid = (int)(need < dev.sms ? (need > 0 ? need : 1) : dev.sms);
         if (gsf_in == nullptr) {

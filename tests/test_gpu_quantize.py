@@ -142,3 +142,20 @@ def test_format_conversions_exhaustive(oracle):
             gs = to_np(sc)[keep]
             bads = np.flatnonzero(gs != os_)
             assert bads.size == 0, f"scale differs for {vk[bads[:6]]}: {gs[bads[:6]]} vs {os_[bads[:6]]}"
+
+
+@pytest.mark.parametrize("group", [0, 128])
+@pytest.mark.parametrize("rows", [4096, 14208, 14336])
+def test_dynamic_single_pass_capacity_edge(oracle, group, rows):
+    """A dynamic-scale call that fits on chip takes the single-pass kernel (up to 14.5 M
+    values on 148 SMs: 14208 x 1024 is exactly the capacity); 14336 x 1024 is just past it
+    and takes the two passes.  Both bit for bit against the oracle."""
+    K = 1024
+    x = W.with_outliers((rows, K), 0.005, 30.0, W._gen(rows + group, "cpu"), "cpu")
+    p, sf, g = nv.nvfp4_quantize(x.to(DEV), group, None)
+    torch.cuda.synchronize()
+    assert nv.last_device_status() == nv.OK
+    xr = oracle.hadamard_rotate(W.to_u16(x), group) if group else W.to_u16(x)
+    op, osf, og = oracle.quantize(xr)
+    assert float(g.item()) == og
+    assert np.array_equal(to_np(p), op) and np.array_equal(to_np(sf), osf)
