@@ -52,8 +52,9 @@ constexpr int SMEM_SFA = 4 * 512;       // four K=64 scale chunks for 128 rows
 constexpr int SMEM_SFB = 8 * 512;       // the same for 256 rows (two 128-row tiles)
 constexpr int STG_BYTES = 32 * 64;      // one 32 x 32 bf16 staging tile
 constexpr int SMEM_STG = EPI_WARPS * 2 * STG_BYTES;
+constexpr int SMEM_BIAS = EPI_WARPS * 256;   // each epilogue warp's 128 bias values of a tile
 constexpr int SMEM_BYTES =
-    1024 + STAGES * (SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB) + SMEM_STG + 256;
+    1024 + STAGES * (SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB) + SMEM_STG + SMEM_BIAS + 256;
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t TMEM_BUF1 = 192;     // second accumulator buffer (overlaps [192, 256))
 constexpr uint32_t TMEM_SF = 448;       // ring of scale-factor slots
@@ -145,7 +146,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     uint8_t* sStg = sB + STAGES * SMEM_B;
     uint8_t* sSFA = sStg + SMEM_STG;
     uint8_t* sSFB = sSFA + STAGES * SMEM_SFA;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SMEM_SFB);
+    uint8_t* sBias = sSFB + STAGES * SMEM_SFB;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sBias + SMEM_BIAS);
     uint64_t* empty = full + STAGES;
     uint64_t* acc_full = empty + STAGES;     // [2]
     uint64_t* acc_free = acc_full + 2;       // [2]
@@ -297,6 +299,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const float alpha = I8 ? 0.0f : *p.alpha;
         const float qgsf = QOUT ? *p.q_gsf : 0.0f;
         uint8_t* stg = sStg + (warp - 2) * 2 * STG_BYTES;
+        uint32_t* sbias = reinterpret_cast<uint32_t*>(sBias + (warp - 2) * 256);
         int stg_sel = 0;
         int it = 0;
         bool ok = true;
@@ -305,6 +308,23 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             tile_coords(p, tile, m_blk, n_blk);
             const int b = it & 1;
             const uint32_t use = (uint32_t)(it >> 1);
+            // The bias of this warp's 128 columns goes to shared memory before the
+            // accumulator wait, so its global-load latency stays off the drain path
+            // (columns past N repeat the last bias; they are never stored).
+            const int n_half = n_blk * BN + half * 128;
+            if (p.bias) {
+                const int n = n_half + 4 * lane;
+                uint2 v;
+                if (n + 4 <= p.N) {
+                    v = *reinterpret_cast<const uint2*>(p.bias + n);
+                } else {
+                    v.x = (uint32_t)p.bias[min(n, p.N - 1)] | ((uint32_t)p.bias[min(n + 1, p.N - 1)] << 16);
+                    v.y = (uint32_t)p.bias[min(n + 2, p.N - 1)] | ((uint32_t)p.bias[min(n + 3, p.N - 1)] << 16);
+                }
+                __syncwarp();   // every lane is done with the previous tile's bias
+                reinterpret_cast<uint2*>(sbias)[lane] = v;
+                __syncwarp();
+            }
             if (!mbar_wait_bounded(&acc_full[b], use & 1, abort_flag, p.status, p.budget_ns)) {
                 ok = false;
                 break;
@@ -318,22 +338,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             const float sx_row = (I8 && row0 + lane < p.M) ? p.sx[row0 + lane] : 0.0f;
             // bf16(alpha * acc + bias) of one 32-column chunk, as 16 bf16 pairs
             auto make_words = [&](const uint32_t (&r)[32], int n0, uint32_t (&packed)[16]) {
-                // the bias as 16 bf16 pairs, widened pair by pair below
+                // the bias as 16 bf16 pairs (shared-memory broadcast), widened pair by pair below
                 uint32_t bw[16];
                 if (p.bias) {
-                    if (n0 + 32 <= p.N) {
-                        const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0);
+                    const uint4* bp = reinterpret_cast<const uint4*>(sbias + (n0 - n_half) / 2);
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const uint4 w = bp[q4];
-                            bw[4 * q4] = w.x; bw[4 * q4 + 1] = w.y;
-                            bw[4 * q4 + 2] = w.z; bw[4 * q4 + 3] = w.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            bw[j] = (uint32_t)p.bias[min(n0 + 2 * j, p.N - 1)] |
-                                    ((uint32_t)p.bias[min(n0 + 2 * j + 1, p.N - 1)] << 16);
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const uint4 w = bp[q4];
+                        bw[4 * q4] = w.x; bw[4 * q4 + 1] = w.y;
+                        bw[4 * q4 + 2] = w.z; bw[4 * q4 + 3] = w.w;
                     }
                 }
 #pragma unroll

@@ -90,9 +90,6 @@ __device__ __forceinline__ void bfly2(float2& a, float2& b) {
     b = d;
 }
 
-// Rotates every g-group of the unit in place (the values stay bf16 words).  Values are
-// held as pairs (2k, 2k+1) of a chunk, so the h = 1 stage works inside a pair and all
-// later stages on whole pairs.
 // rn(lo + hi) and rn(lo - hi) of one bf16 pair, with hi widened to fp32 and lo used
 // as a bf16 operand of the mixed-precision add and subtract (exact widening, one
 // rounding each, so both equal the plain fp32 results, signed zeros included).
@@ -105,13 +102,14 @@ __device__ __forceinline__ float2 pair_sum_diff(uint32_t w) {
     return make_float2(s, d);
 }
 
-// Rotates every g-group of the unit in place (the values stay bf16 words).  Values are
+// The butterfly stages of a unit's g-groups in fp32, up to but not including the
+// in-lane stage that is LOCAL_END local chunks apart (G / 16: every stage).  Values are
 // held as pairs (2k, 2k+1) of a chunk, so the h = 1 stage works inside a pair and all
 // later stages on whole pairs.
-template <int G>
-__device__ __forceinline__ void rotate_unit(uint4 (&w)[UnitShape<G>::NCT], int h, float hscale) {
+template <int G, int LOCAL_END>
+__device__ __forceinline__ void butterfly(const uint4 (&w)[UnitShape<G>::NCT], int h,
+                                          float2 (&v)[UnitShape<G>::NCT][4]) {
     constexpr int NCT = UnitShape<G>::NCT;
-    float2 v[NCT][4];
 #pragma unroll
     for (int i = 0; i < NCT; ++i) {
         // h = 1: inside each pair, straight from the bf16 words
@@ -139,12 +137,21 @@ __device__ __forceinline__ void rotate_unit(uint4 (&w)[UnitShape<G>::NCT], int h
         }
     // h = 16, 32, 64: chunks two, four, eight apart = local chunks 1, 2, 4 apart
 #pragma unroll
-    for (int s = 1; s < G / 16; s *= 2)
+    for (int s = 1; s < LOCAL_END; s *= 2)
 #pragma unroll
         for (int i = 0; i < NCT; ++i)
             if ((i & s) == 0)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) bfly2(v[i][k], v[i + s][k]);
+}
+
+// Rotates every g-group of the unit in place (the values stay bf16 words): the whole
+// butterfly, the 1/sqrt(g) scale and the rounding to bf16.
+template <int G>
+__device__ __forceinline__ void rotate_unit(uint4 (&w)[UnitShape<G>::NCT], int h, float hscale) {
+    constexpr int NCT = UnitShape<G>::NCT;
+    float2 v[NCT][4];
+    butterfly<G, G / 16>(w, h, v);
     const float2 hs = make_float2(hscale, hscale);
 #pragma unroll
     for (int i = 0; i < NCT; ++i) {
@@ -154,6 +161,40 @@ __device__ __forceinline__ void rotate_unit(uint4 (&w)[UnitShape<G>::NCT], int h
         w[i] = make_uint4(bf16x2_rn(g[0].x, g[0].y), bf16x2_rn(g[1].x, g[1].y),
                           bf16x2_rn(g[2].x, g[2].y), bf16x2_rn(g[3].x, g[3].y));
     }
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Running maximum of |v| over the unit's rotated values before the 1/sqrt(g) scale and
+// the bf16 rounding (G >= 32, where the last stage is in-lane).  The last stage maps
+// (a, b) to rn(a + b) and rn(a - b); one of |a + b|, |a - b| is |a| + |b| exactly and
+// rounding is monotone and odd, so the larger magnitude of the two outputs is
+// rn(|a| + |b|).  The rotated bf16 value is bf16(rn(v * hscale)), also monotone in |v|,
+// so the bf16 amax of the unit is bf16(rn(m * hscale)) of this maximum m.
+template <int G>
+__device__ __forceinline__ float rotate_amax(const uint4 (&w)[UnitShape<G>::NCT], int h, float m) {
+    static_assert(G >= 32, "the last stage must be in-lane");
+    constexpr int NCT = UnitShape<G>::NCT;
+    constexpr int S = G / 32;
+    float2 v[NCT][4];
+    butterfly<G, S>(w, h, v);
+#pragma unroll
+    for (int i = 0; i < NCT; ++i)
+        if ((i & S) == 0)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                m = max3(m, __fadd_rn(fabsf(v[i][k].x), fabsf(v[i + S][k].x)),
+                         __fadd_rn(fabsf(v[i][k].y), fabsf(v[i + S][k].y)));
+    return m;
+}
+
+// bf16(rn(m * hscale)) as fp32: the amax of the rotated bf16 values (see rotate_amax).
+__device__ __forceinline__ float rotated_amax_bf16(float m, float hscale) {
+    return bf16lo(bf16x2_rn(__fmul_rn(m, hscale), 0.0f));
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -298,7 +339,8 @@ __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
 
     float gsf = 0.0f;
     if constexpr (MODE == 1) gsf = encode_prologue<kThreads>(p, red, &s_gsf, inv_tab);
-    uint32_t tmax = 0u;
+    uint32_t tmax = 0u;       // packed bf16 maxima (G < 32)
+    float fmax_rot = 0.0f;    // pre-scale rotated maximum (G >= 32)
 
     // (row, u) of this lane's unit, advanced by the grid stride without dividing again
     const int64_t stride = n_warps * 16;
@@ -326,6 +368,10 @@ __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
                        ? (MODE == 2 ? ld_plain(src + c * 8) : ld_stream(src + c * 8))
                        : make_uint4(0, 0, 0, 0);
         }
+        if constexpr (MODE == 0 && G >= 32) {
+            fmax_rot = rotate_amax<G>(w, h, fmax_rot);
+            continue;
+        }
         if constexpr (G > 0) rotate_unit<G>(w, h, p.hscale);
 
         if constexpr (MODE == 2) {
@@ -343,7 +389,8 @@ __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
         }
     }
     if constexpr (MODE == 0) {
-        const float m = block_max(absmax_of_pair(tmax), red);
+        const float mine = G >= 32 ? rotated_amax_bf16(fmax_rot, p.hscale) : absmax_of_pair(tmax);
+        const float m = block_max(mine, red);
         if (threadIdx.x == 0) p.partials_out[blockIdx.x] = m;
     }
 }
@@ -449,7 +496,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     }
 
     const int pair = lane >> 1;
-    uint32_t tmax = 0u;
+    uint32_t tmax = 0u;       // packed bf16 maxima (G < 32)
+    float fmax_rot = 0.0f;    // pre-scale rotated maximum (G >= 32)
     uint32_t k = 0;
     for (uint32_t item = first; item < t.n_items; item += stride, ++k) {
         const int s = (int)(k % kSlots);
@@ -484,17 +532,21 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             const bool active = unit < t.total_units;
             const uint32_t row = fast_div(unit, t.upr_div);
             const int64_t e0 = (int64_t)(unit - row * t.upr) * E;
-            if constexpr (G > 0) rotate_unit<G>(w[sub], h, p.hscale);
-            if constexpr (MODE == 0) {
+            if constexpr (MODE == 0 && G >= 32) {
+                fmax_rot = rotate_amax<G>(w[sub], h, fmax_rot);
+            } else if constexpr (MODE == 0) {
+                if constexpr (G > 0) rotate_unit<G>(w[sub], h, p.hscale);
 #pragma unroll
                 for (int i = 0; i < NCT; ++i) tmax = absmax2_bf16(tmax, absmax_word4(w[sub][i]));
             } else {
+                if constexpr (G > 0) rotate_unit<G>(w[sub], h, p.hscale);
                 encode_unit<G>(w[sub], h, gsf, inv_tab, p, (int64_t)row, e0, E, active, active);
             }
         }
     }
     if constexpr (MODE == 0) {
-        const float mx = block_max(absmax_of_pair(tmax), red);
+        const float mine = G >= 32 ? rotated_amax_bf16(fmax_rot, p.hscale) : absmax_of_pair(tmax);
+        const float mx = block_max(mine, red);
         if (threadIdx.x == 0) p.partials_out[blockIdx.x] = mx;
     }
     // after a timeout, let this warp's loads still in flight land before the CTA exits

@@ -159,3 +159,28 @@ def test_dynamic_single_pass_capacity_edge(oracle, group, rows):
     op, osf, og = oracle.quantize(xr)
     assert float(g.item()) == og
     assert np.array_equal(to_np(p), op) and np.array_equal(to_np(sf), osf)
+
+
+@pytest.mark.parametrize("group", [16, 32, 64, 128])
+def test_dynamic_two_pass_rotated(oracle, group):
+    """Past the single-pass capacity (16384 x 1024 = 16.8 M values) a dynamic call runs the
+    amax pass, then the encode pass.  With g >= 32 the amax pass stops before the last
+    butterfly stage, keeps max(|a| + |b|) of its operand pairs, and scales and rounds that
+    maximum once; the global scale must still equal the oracle's bit for bit."""
+    rows, K = 16384, 1024
+    x = W.with_outliers((rows, K), 0.005, 30.0, W._gen(rows * 3 + group, "cpu"), "cpu")
+    check(oracle, x, group, None)
+
+
+@pytest.mark.parametrize("sign", [1.0, -1.0])
+@pytest.mark.parametrize("R,K", [(3, 96), (257, 160)])
+def test_dynamic_amax_last_stage_branch(oracle, sign, R, K):
+    """The largest rotated value comes out of the last stage's sum (sign +1) or its
+    difference (sign -1): g = 32 over [1, 0 x 15, sign, 0 x 15] gives halves of all ones and
+    all `sign`, so a + b or a - b is 2 and the other is 0.  K % 64 != 0 keeps the plain-load
+    kernels (amax pass, then encode pass)."""
+    g = torch.Generator().manual_seed(int(K + 10 * sign))
+    x = torch.randn(R, K, generator=g) * 1e-3
+    x[1, 32] = 1.0
+    x[1, 48] = sign
+    check(oracle, x.to(torch.bfloat16), 32, None)
