@@ -145,7 +145,9 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t 
  *   K % 64 == 0 (32-byte packed rows keep the tensor-map rows aligned and match the
  *   128x4 scale tiling); M, N >= 0, each below 2^31.
  * y[m,n] = bf16(fp32(alpha * acc) + bias[n]), acc = the fp32 tensor-core sum of
- * (e2m1_a * e4m3_a) * (e2m1_b * e4m3_b) over k.
+ * (e2m1_a * e4m3_a) * (e2m1_b * e4m3_b) over k.  When the 128 x 256 output tiles
+ * fill at most half of the SMs (small M), K is split over a thread-block cluster and
+ * the partial sums are added in a fixed order, so results are deterministic either way.
  * Errors: INVALID_ARG, SHAPE, ALIGN, DEVICE, CUDA.
  */
 NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,

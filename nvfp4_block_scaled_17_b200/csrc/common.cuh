@@ -377,6 +377,38 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// --- thread-block clusters -----------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Every thread of every CTA of the cluster arrives and waits (per-thread form, no
+// warp convergence required): the shared-memory writes before it are visible to the
+// whole cluster after it.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile(
+        "barrier.cluster.arrive.release;\n\t"
+        "barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// The address of the same shared-memory offset in the CTA of cluster rank `rank`.
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 // Shared-memory matrix descriptor (sm_100 version 1): K-major, 128-byte swizzle,
 // 8-row core groups 1024 bytes apart (SBO), leading offset unused.
 __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t smem_addr) {

@@ -28,11 +28,20 @@
 // first and releases it, so the MMAs of the next tile start while the rest of the
 // previous accumulator is still being stored.
 //
+// Small grids (at most half as many tiles as SMs, e.g. M <= 128 at N = 5120) take the
+// split-K build instead: a cluster of S CTAs per tile, CTA r of the cluster running the
+// same pipeline over its share of the K tiles; the raw fp32 partial tile goes to that
+// CTA's own (now idle) stage buffers, and after a cluster barrier rank r sums its share
+// of the rows over all S partials (distributed shared memory, rank order) and applies
+// alpha and the bias.
+//
 // Every wait is bounded (globaltimer); on expiry the kernel records
 // NVFP4_ERR_TIMEOUT, drains its own copies and MMAs, frees tensor memory and exits.
 // No load uses cluster multicast.
 #include "common.cuh"
 #include "kernels.h"
+
+#include <atomic>
 
 #include <cudaTypedefs.h>
 
@@ -81,6 +90,7 @@ struct GemmParams {
     int sf_row_tiles_b;        // ceil(N / 128)
     int tma_store;             // 1: y through the tensor map (N % 8 == 0)
     int n_fast;                // tile order: 1 = consecutive tiles walk N (B re-read from L2)
+    int splits;                // split-K build: CTAs (one cluster) sharing the K range of a tile
     // quantized output (the NVFP4 input of the next linear), when the kernel is built for it
     uint8_t* q_packed;         // [M, N/2]
     uint8_t* q_sf;             // 128x4 scales of an [M, N] operand
@@ -134,7 +144,7 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& 
     }
 }
 
-template <bool QOUT, bool I8>
+template <bool QOUT, bool I8, bool SPLITK>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
@@ -180,6 +190,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const uint32_t tmem = *tmem_holder;
 
     const int num_tiles = p.m_blocks * p.n_blocks;
+    // This CTA's work: whole tiles, persistent over the grid; or (split-K) the K range
+    // [kt_begin, kt_end) of the one tile that its cluster shares.
+    const int splits = SPLITK ? p.splits : 1;
+    const int rank = SPLITK ? (int)cluster_rank() : 0;
+    const int tile_first = SPLITK ? (int)blockIdx.x / splits : (int)blockIdx.x;
+    const int tile_step = SPLITK ? num_tiles : (int)gridDim.x;
+    const int kt_begin = SPLITK ? rank * p.k_tiles / splits : 0;
+    const int kt_end = SPLITK ? (rank + 1) * p.k_tiles / splits : p.k_tiles;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -189,11 +207,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             uint32_t phase = 0;
             uint32_t issued = 0, issued_phase = 0;   // per-stage bit masks
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            for (int tile = tile_first; ok && tile < num_tiles; tile += tile_step) {
                 int m_blk, n_blk;
                 tile_coords(p, tile, m_blk, n_blk);
                 const int sfb_tiles = (2 * n_blk + 1 < p.sf_row_tiles_b) ? 2 : 1;
-                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                for (int kt = kt_begin; kt < kt_end; ++kt) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status,
                                            p.budget_ns)) {
                         ok = false;
@@ -236,7 +254,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             bool ok = true;
             int it = 0;
             int sf_slot = 0;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+            for (int tile = tile_first; ok && tile < num_tiles; tile += tile_step, ++it) {
                 const int b = it & 1;
                 const uint32_t use = (uint32_t)(it >> 1);
                 // buffer b fully drained (tile it-2) and the shared columns drained (tile it-1)
@@ -249,7 +267,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 }
                 tc_fence_after();
                 const uint32_t acc = tmem + (b ? TMEM_BUF1 : 0u);
-                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                for (int kt = kt_begin; kt < kt_end; ++kt) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status,
                                            p.budget_ns)) {
                         ok = false;
@@ -264,7 +282,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     for (int kk = 0; kk < steps; ++kk) {
                         if constexpr (I8) {
                             mma_i8(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
-                                   sdesc_kmajor_sw128(b0 + 32 * kk), IDESC_I8, (kt | kk) != 0);
+                                   sdesc_kmajor_sw128(b0 + 32 * kk), IDESC_I8,
+                                   kt > kt_begin || kk > 0);
                         } else {
                             const uint32_t sfa_t = tmem + TMEM_SF + 12u * (uint32_t)sf_slot;
                             const uint32_t sfb_t = sfa_t + 4;
@@ -273,7 +292,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                             tc_copy_sf(sfb_t + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
                             mma_nvf4(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
                                      sdesc_kmajor_sw128(b0 + 32 * kk), IDESC, sfa_t, sfb_t,
-                                     (kt | kk) != 0);
+                                     kt > kt_begin || kk > 0);
                             if (++sf_slot == SF_SLOTS) sf_slot = 0;
                         }
                     }
@@ -303,7 +322,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         int stg_sel = 0;
         int it = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+        for (int tile = tile_first; ok && tile < num_tiles; tile += tile_step, ++it) {
             int m_blk, n_blk;
             tile_coords(p, tile, m_blk, n_blk);
             const int b = it & 1;
@@ -421,6 +440,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&acc_free[b]);
                 }
+                if constexpr (SPLITK) {
+                    // the raw fp32 partial into this CTA's partial tile (the stage buffers,
+                    // idle now): row-major 1 KiB rows, 16-byte granule g of row r at
+                    // g ^ (r & 7), so eight lanes of a store phase hit eight bank groups
+                    const int row = quad * 32 + lane;
+                    uint8_t* prow = smem + row * 1024;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        *reinterpret_cast<uint4*>(prow + (((c0 * 8 + j) ^ (row & 7)) << 4)) =
+                            make_uint4(r0[4 * j], r0[4 * j + 1], r0[4 * j + 2], r0[4 * j + 3]);
+                        *reinterpret_cast<uint4*>(prow + (((c1 * 8 + j) ^ (row & 7)) << 4)) =
+                            make_uint4(r1[4 * j], r1[4 * j + 1], r1[4 * j + 2], r1[4 * j + 3]);
+                    }
+                    continue;
+                }
                 const int n00 = n_blk * BN + c0 * 32, n01 = n_blk * BN + c1 * 32;
                 uint32_t w0[16], w1[16];
                 if (n00 < p.N) make_words(r0, n00, w0);   // warp-uniform
@@ -458,6 +492,53 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (SPLITK) {
+        // Every thread of the cluster gets here after bounded work (all waits above are
+        // bounded), so the two cluster barriers cannot hang.  Rank r then sums rows
+        // [r R / S, (r + 1) R / S) of the S partial tiles in rank order over distributed
+        // shared memory and stores them; the second barrier keeps every partial alive
+        // until all ranks have read it.
+        cluster_sync_all();
+        if (warp >= 2) {
+            int m_blk, n_blk;
+            tile_coords(p, tile_first, m_blk, n_blk);
+            const int rows = min(BM, p.M - m_blk * BM);
+            const int r_lo = rank * rows / splits, r_hi = (rank + 1) * rows / splits;
+            const uint32_t part = smem_u32(smem);
+            const float alpha = *p.alpha;
+            for (int idx = threadIdx.x - 64; idx < (r_hi - r_lo) * 64; idx += 32 * EPI_WARPS) {
+                const int row = r_lo + (idx >> 6), g = idx & 63;
+                const int col = n_blk * BN + 4 * g;
+                if (col >= p.N) continue;
+                const uint32_t off = part + (uint32_t)(row * 1024 + ((g ^ (row & 7)) << 4));
+                float4 acc = ld_dsmem_f4(dsmem_addr(off, 0));
+                for (int r = 1; r < splits; ++r) {
+                    const float4 v = ld_dsmem_f4(dsmem_addr(off, (uint32_t)r));
+                    acc.x = __fadd_rn(acc.x, v.x);
+                    acc.y = __fadd_rn(acc.y, v.y);
+                    acc.z = __fadd_rn(acc.z, v.z);
+                    acc.w = __fadd_rn(acc.w, v.w);
+                }
+                float v[4] = {__fmul_rn(alpha, acc.x), __fmul_rn(alpha, acc.y),
+                              __fmul_rn(alpha, acc.z), __fmul_rn(alpha, acc.w)};
+                if (p.bias) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        v[j] = __fadd_rn(v[j], __uint_as_float((uint32_t)p.bias[min(col + j, p.N - 1)] << 16));
+                }
+                const uint32_t lo = bf16x2_bits(v[0], v[1]), hi = bf16x2_bits(v[2], v[3]);
+                uint16_t* yp = p.y + (size_t)(m_blk * BM + row) * p.N + col;
+                if ((p.N & 3) == 0 && col + 4 <= p.N) {
+                    *reinterpret_cast<uint2*>(yp) = make_uint2(lo, hi);
+                } else {
+                    const uint16_t hv[4] = {(uint16_t)lo, (uint16_t)(lo >> 16), (uint16_t)hi,
+                                            (uint16_t)(hi >> 16)};
+                    for (int j = 0; j < 4 && col + j < p.N; ++j) yp[j] = hv[j];
+                }
+            }
+        }
+        cluster_sync_all();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
@@ -505,6 +586,71 @@ struct QuantOut {
     const float* gsf;
 };
 
+// Split-K build: clusters of `splits` CTAs, one tile per cluster.
+cudaLaunchConfig_t split_k_config(int grid, int splits, cudaStream_t stream,
+                                  cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+bool split_k_attr(int device) {
+    static std::atomic<int> done[64];
+    if (done[device & 63].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(gemm_kernel<false, false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+        return false;
+    done[device & 63].store(1, std::memory_order_release);
+    return true;
+}
+
+// K splits for a grid with too few tiles to fill the SMs: the largest S <= 8 (a portable
+// cluster) with S <= ceil(K / 256) and tiles * S <= SMs whose clusters are all resident
+// at once (cudaOccupancyMaxActiveClusters, cached per device and S); 1 = no split.
+int choose_splits(int tiles, int k_tiles, const DeviceInfo& dev) {
+    if (tiles * 2 > dev.sms || k_tiles < 2) return 1;
+    if (!split_k_attr(dev.device)) return 1;
+    static std::atomic<int> cap[64][9];   // max active clusters + 1 (0 = not queried yet)
+    const int smax = min(8, min(k_tiles, dev.sms / tiles));
+    for (int sp = smax; sp >= 2; --sp) {
+        int c = cap[dev.device & 63][sp].load(std::memory_order_relaxed) - 1;
+        if (c < 0) {
+            cudaLaunchAttribute attr[1];
+            const cudaLaunchConfig_t cfg = split_k_config(sp * tiles, sp, nullptr, attr);
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<false, false, true>, &cfg) !=
+                cudaSuccess) {
+                (void)cudaGetLastError();
+                n = 0;
+            }
+            c = n;
+            cap[dev.device & 63][sp].store(c + 1, std::memory_order_relaxed);
+        }
+        if (c >= tiles) return sp;
+    }
+    return 1;
+}
+
+nvfp4_status launch_split_k(const CUtensorMap& mapA, const CUtensorMap& mapB,
+                            const CUtensorMap& mapY, const GemmParams& p, int grid, int splits,
+                            cudaStream_t stream) {
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = split_k_config(grid, splits, stream, attr);
+    if (cudaLaunchKernelEx(&cfg, gemm_kernel<false, false, true>, mapA, mapB, mapY, p) !=
+        cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
+
 // One launcher for the three builds of the kernel: NVFP4 (sfa/sfb = 128x4 scales,
 // alpha), NVFP4 with the quantized output, and int8 (sfa/sfb unused; sx/sw = fp32 row
 // scales of A and B).
@@ -532,8 +678,8 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
 
     static bool attr_set[64] = {false};
     if (!attr_set[dev.device & 63]) {
-        if (cudaFuncSetAttribute(gemm_kernel<QOUT, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemm_kernel<QOUT, I8, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         attr_set[dev.device & 63] = true;
     }
@@ -555,6 +701,7 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
     p.sf_row_tiles_b = (int)((N + 127) / 128);
     p.tma_store = tma_store ? 1 : 0;
     p.n_fast = (N <= M) ? 1 : 0;
+    p.splits = 1;
     if (QOUT) {
         p.q_packed = q->packed;
         p.q_sf = q->sf;
@@ -565,8 +712,15 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
     p.budget_ns = 4000000000ull;   // 4 s
 
     const int tiles = p.m_blocks * p.n_blocks;
+    if constexpr (!QOUT && !I8) {
+        const int splits = choose_splits(tiles, p.k_tiles, dev);
+        if (splits > 1) {
+            p.splits = splits;
+            return launch_split_k(mapA, mapB, mapY, p, tiles * splits, splits, stream);
+        }
+    }
     const int grid = tiles < dev.sms ? tiles : dev.sms;
-    gemm_kernel<QOUT, I8><<<grid, THREADS, SMEM_BYTES, stream>>>(mapA, mapB, mapY, p);
+    gemm_kernel<QOUT, I8, false><<<grid, THREADS, SMEM_BYTES, stream>>>(mapA, mapB, mapY, p);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 

@@ -57,6 +57,54 @@ def test_gemm_parity(oracle, M, N, K, bias):
     run_gemm_case(oracle, M, N, K, bias, seed=M * 31 + N * 7 + K)
 
 
+@pytest.mark.parametrize("M,N,K,rows", [
+    (16, 5120, 5120, None),      # the M-sweep's decode shapes: 20 tiles on 148 SMs
+    (128, 5120, 5120, 24),
+    (7, 2050, 768, None),        # N % 4 != 0: element-wise stores of the reduced rows
+    (1, 64, 4096, None),
+    (130, 520, 1536, None),      # two row blocks, ragged N and M
+])
+def test_gemm_split_k(oracle, M, N, K, rows):
+    """Grids with at most half as many tiles as SMs split K over a cluster of CTAs and
+    reduce the partial tiles over distributed shared memory."""
+    sel = None if rows is None else sample_rows(M, rows, seed=M + N)
+    run_gemm_case(oracle, M, N, K, bias=True, seed=M * 13 + N + K, rows=sel)
+
+
+def test_gemm_split_k_deterministic_and_graph_capturable():
+    """The split-K reduction adds the partial tiles in a fixed order, so repeated calls
+    agree bit for bit; the call also replays from a CUDA graph with the same result."""
+    M, N, K = 16, 5120, 5120
+    g = torch.Generator(device="cpu").manual_seed(11)
+    xp = torch.randint(0, 256, (M, K // 2), generator=g, dtype=torch.uint8).to(DEV)
+    wp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8).to(DEV)
+    # scale bytes 0x30..0x3f (E4M3 0.5 .. 0.94): finite, positive
+    xsf = (0x30 + torch.randint(0, 16, (nv.nvfp4_scale_bytes(M, K),), generator=g)).to(torch.uint8).to(DEV)
+    wsf = (0x30 + torch.randint(0, 16, (nv.nvfp4_scale_bytes(N, K),), generator=g)).to(torch.uint8).to(DEV)
+    al = torch.tensor([1e-3], device=DEV)
+    bias = (torch.randn(N, generator=g) * 0.01).to(torch.bfloat16).to(DEV)
+    y1 = nv.nvfp4_gemm(xp, xsf, wp, wsf, al, bias, M, N, K)
+    y2 = nv.nvfp4_gemm(xp, xsf, wp, wsf, al, bias, M, N, K)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    y3 = torch.empty_like(y1)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        nv.nvfp4_gemm(xp, xsf, wp, wsf, al, bias, M, N, K, out=y3)   # warm-up on the stream
+        torch.cuda.synchronize()
+        y3.zero_()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=s):
+            nv.nvfp4_gemm(xp, xsf, wp, wsf, al, bias, M, N, K, out=y3)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert nv.last_device_status() == nv.OK
+    assert torch.equal(y1.view(torch.int16), y3.view(torch.int16))
+    del graph
+
+
 def test_gemm_vit_qkv_full_size(oracle):
     """ViT block qkv projection: [32768, 1024] x [3072, 1024]^T, sampled rows."""
     run_gemm_case(oracle, 32768, 3072, 1024, True, seed=11, rows=sample_rows(32768, 96))
