@@ -46,10 +46,10 @@ METRIC = "nvfp4_linear TFLOPS (% of dense FP4 peak); quantizer GB/s (% of HBM)"
 # profiles/vit_block_step_launches.md, valid only for the kernel sources it was taken on
 # (sha256 prefix); reported as null once a source has changed.
 MEASURED_TRAFFIC = {
-    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "eec3e6d02cf3a787",
-             "bytes_per_step": 530.4e6},
-    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "aec233f10454b338",
-              "bytes_per_step": 959.3e6},
+    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "94843ccec54eb473",
+             "bytes_per_step": 530.1e6},
+    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "89c3e8f04aaae56e",
+              "bytes_per_step": 959.2e6},
 }
 
 
