@@ -46,10 +46,10 @@ METRIC = "nvfp4_linear TFLOPS (% of dense FP4 peak); quantizer GB/s (% of HBM)"
 # profiles/vit_block_step_launches.md, valid only for the kernel sources it was taken on
 # (sha256 prefix); reported as null once a source has changed.
 MEASURED_TRAFFIC = {
-    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "94843ccec54eb473",
-             "bytes_per_step": 530.1e6},
-    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "89c3e8f04aaae56e",
-              "bytes_per_step": 959.2e6},
+    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "4ec0158c7a54741a",
+             "bytes_per_step": 530.3e6},
+    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "6de0f6e3f8099c0b",
+              "bytes_per_step": 959.1e6},
 }
 
 
@@ -199,23 +199,29 @@ def run_step(layers, dynamic: bool, events=None):
 
 
 def timed_steps(layers, dynamic, steps, warmup, dist_on):
+    """The K timed steps with nothing between the launches (start/stop events only, so
+    consecutive kernels can overlap their launch and set-up), then the same K steps once
+    more with an event around every launch for the per-kernel durations."""
     for _ in range(warmup):
         run_step(layers, dynamic)
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in layers]
-           for _ in range(steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     start.record()
-    for k in range(steps):
-        run_step(layers, dynamic, evs[k])
+    for _ in range(steps):
+        run_step(layers, dynamic)
     stop.record()
     torch.cuda.synchronize()
     if dist_on:
         torch.distributed.barrier()
     total_ms = start.elapsed_time(stop)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in layers]
+           for _ in range(steps)]
+    for k in range(steps):
+        run_step(layers, dynamic, evs[k])
+    torch.cuda.synchronize()
     q_ms = [sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(steps)) / steps
             for i in range(len(layers))]
     g_ms = [sum(evs[k][i][1].elapsed_time(evs[k][i][2]) for k in range(steps)) / steps

@@ -377,6 +377,21 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// --- programmatic dependent launch ------------------------------------------------------
+// A kernel launched with programmatic stream serialization may start while the kernel
+// before it on the stream is finishing.  It sets up its shared and tensor memory, then
+// waits here until that kernel has completed and its memory is visible; nothing before
+// this wait reads or writes global memory.  (A no-op for an ordinary launch.)
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets the next kernel on the stream be scheduled as SMs free up (it still runs its own
+// griddep_wait before touching memory).
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // --- thread-block clusters -----------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;

@@ -188,6 +188,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    griddep_wait();
+    griddep_launch_dependents();
 
     const int num_tiles = p.m_blocks * p.n_blocks;
     // This CTA's work: whole tiles, persistent over the grid; or (split-K) the K range
@@ -588,7 +590,7 @@ struct QuantOut {
 
 // Split-K build: clusters of `splits` CTAs, one tile per cluster.
 cudaLaunchConfig_t split_k_config(int grid, int splits, cudaStream_t stream,
-                                  cudaLaunchAttribute* attr) {
+                                  cudaLaunchAttribute* attr, bool pdl = false) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3(THREADS, 1, 1);
@@ -598,8 +600,10 @@ cudaLaunchConfig_t split_k_config(int grid, int splits, cudaStream_t stream,
     attr[0].val.clusterDim.x = (unsigned)splits;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     return cfg;
 }
 
@@ -624,7 +628,7 @@ int choose_splits(int tiles, int k_tiles, const DeviceInfo& dev) {
     for (int sp = smax; sp >= 2; --sp) {
         int c = cap[dev.device & 63][sp].load(std::memory_order_relaxed) - 1;
         if (c < 0) {
-            cudaLaunchAttribute attr[1];
+            cudaLaunchAttribute attr[2];
             const cudaLaunchConfig_t cfg = split_k_config(sp * tiles, sp, nullptr, attr);
             int n = 0;
             if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<false, false, true>, &cfg) !=
@@ -643,8 +647,8 @@ int choose_splits(int tiles, int k_tiles, const DeviceInfo& dev) {
 nvfp4_status launch_split_k(const CUtensorMap& mapA, const CUtensorMap& mapB,
                             const CUtensorMap& mapY, const GemmParams& p, int grid, int splits,
                             cudaStream_t stream) {
-    cudaLaunchAttribute attr[1];
-    const cudaLaunchConfig_t cfg = split_k_config(grid, splits, stream, attr);
+    cudaLaunchAttribute attr[2];
+    const cudaLaunchConfig_t cfg = split_k_config(grid, splits, stream, attr, true);
     if (cudaLaunchKernelEx(&cfg, gemm_kernel<false, false, true>, mapA, mapB, mapY, p) !=
         cudaSuccess)
         return NVFP4_ERR_CUDA;
@@ -720,8 +724,10 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
         }
     }
     const int grid = tiles < dev.sms ? tiles : dev.sms;
-    gemm_kernel<QOUT, I8, false><<<grid, THREADS, SMEM_BYTES, stream>>>(mapA, mapB, mapY, p);
-    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+    if (launch_pdl(gemm_kernel<QOUT, I8, false>, (unsigned)grid, THREADS, SMEM_BYTES, stream, mapA,
+                   mapB, mapY, p) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
 }
 
 }  // namespace

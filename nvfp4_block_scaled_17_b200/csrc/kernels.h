@@ -10,6 +10,25 @@
 namespace nvfp4 {
 
 // Cached per-device facts (multiprocessor count, compute capability).
+// Launch with programmatic stream serialization (the kernel overlaps its set-up with the
+// tail of the previous kernel on the stream and runs griddep_wait() before any global
+// memory access).  Used for the persistent kernels, whose grid is resident at once.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block,
+                              size_t smem, cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(block, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 struct DeviceInfo {
     int device = -1;
     int sms = 0;

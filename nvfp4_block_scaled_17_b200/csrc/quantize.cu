@@ -464,6 +464,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         for (int s = 0; s < kSlots; ++s) mbar_init(&full[warp * kSlots + s], 1);
     fence_barrier_init();
     __syncthreads();
+    griddep_wait();
+    griddep_launch_dependents();
 
     float gsf = 0.0f;
     if constexpr (MODE == 1) {
@@ -790,8 +792,10 @@ nvfp4_status launch_tma_unit(const CUtensorMap& map, const UnitParams& p, const 
             return NVFP4_ERR_CUDA;
         attr_set[device] = true;
     }
-    tma_unit_kernel<G, MODE><<<grid, kTmaThreads, smem, stream>>>(map, p, t, status);
-    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+    if (launch_pdl(tma_unit_kernel<G, MODE>, (unsigned)grid, kTmaThreads, smem, stream, map, p, t,
+                   status) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
 }
 
 template <int MODE>
