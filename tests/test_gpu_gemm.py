@@ -30,7 +30,11 @@ def sample_rows(M: int, n: int, seed: int = 0) -> np.ndarray:
     return np.array(sorted(pick), dtype=np.int64)
 
 
-def run_gemm_case(oracle, M, N, K, bias: bool, seed: int, rows=None):
+def run_gemm_case(oracle, M, N, K, bias: bool, seed: int, rows=None, cols=None):
+    """GPU GEMM against the fp64 oracle on the rows `rows` (all when None) x all columns,
+    and, when `cols` is given, also on all rows x the columns `cols`.  The column check
+    runs the oracle on the transposed product: y^T[cols] = alpha deq(w[cols]) deq(x)^T,
+    then adds the bias of those columns."""
     x = W.with_outliers((M, K), 0.01, 20.0, W._gen(seed, "cpu"), "cpu")
     w = W.normal((N, K), 0.02, W._gen(seed + 1, "cpu"), "cpu").to(torch.bfloat16)
     b = W.normal((N,), 0.01, W._gen(seed + 2, "cpu"), "cpu").to(torch.bfloat16) if bias else None
@@ -44,7 +48,14 @@ def run_gemm_case(oracle, M, N, K, bias: bool, seed: int, rows=None):
     y64 = oracle.gemm_f64(xp, xsf, wp, wsf, M, N, K, al, None if b is None else W.to_u16(b),
                           rows=rows)
     yg = y if rows is None else y[torch.from_numpy(rows).to(DEV)]
-    return assert_gemm_close(yg, y64, f"gemm M={M} N={N} K={K}")
+    out = assert_gemm_close(yg, y64, f"gemm M={M} N={N} K={K}")
+    if cols is not None:
+        yt64 = oracle.gemm_f64(wp, wsf, xp, xsf, N, M, K, al, None, rows=cols)
+        if b is not None:
+            yt64 = yt64 + b.float().numpy().astype(np.float64)[cols][:, None]
+        yc = y[:, torch.from_numpy(cols).to(DEV)].t().contiguous()
+        assert_gemm_close(yc, yt64, f"gemm M={M} N={N} K={K}, all rows x {len(cols)} columns")
+    return out
 
 
 @pytest.mark.parametrize("M,N,K", [
@@ -106,13 +117,17 @@ def test_gemm_split_k_deterministic_and_graph_capturable():
 
 
 def test_gemm_vit_qkv_full_size(oracle):
-    """ViT block qkv projection: [32768, 1024] x [3072, 1024]^T, sampled rows."""
-    run_gemm_case(oracle, 32768, 3072, 1024, True, seed=11, rows=sample_rows(32768, 96))
+    """ViT block qkv projection: [32768, 1024] x [3072, 1024]^T, 256 sampled rows x all
+    columns and all rows x 256 sampled columns."""
+    run_gemm_case(oracle, 32768, 3072, 1024, True, seed=11, rows=sample_rows(32768, 256),
+                  cols=sample_rows(3072, 256, seed=5))
 
 
 def test_gemm_down_proj_full_size(oracle):
-    """Qwen3-VL down_proj shape with the full K = 25600: [4096, 25600] x [5120, 25600]^T."""
-    run_gemm_case(oracle, 4096, 5120, 25600, False, seed=13, rows=sample_rows(4096, 12))
+    """Qwen3-VL down_proj shape with the full K = 25600: [4096, 25600] x [5120, 25600]^T,
+    256 sampled rows x all columns and all rows x 256 sampled columns."""
+    run_gemm_case(oracle, 4096, 5120, 25600, False, seed=13, rows=sample_rows(4096, 256),
+                  cols=sample_rows(5120, 256, seed=7))
 
 
 def test_gemm_zero_sizes():
