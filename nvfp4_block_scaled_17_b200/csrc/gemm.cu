@@ -91,6 +91,7 @@ struct GemmParams {
     int tma_store;             // 1: y through the tensor map (N % 8 == 0)
     int n_fast;                // tile order: 1 = consecutive tiles walk N (B re-read from L2)
     int splits;                // split-K build: CTAs (one cluster) sharing the K range of a tile
+    int tile_base, tile_count; // the tiles of this launch: [tile_base, tile_base + tile_count)
     // quantized output (the NVFP4 input of the next linear), when the kernel is built for it
     uint8_t* q_packed;         // [M, N/2]
     uint8_t* q_sf;             // 128x4 scales of an [M, N] operand
@@ -191,7 +192,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     griddep_wait();
     griddep_launch_dependents();
 
-    const int num_tiles = p.m_blocks * p.n_blocks;
+    const int num_tiles = p.tile_count;
     // This CTA's work: whole tiles, persistent over the grid; or (split-K) the K range
     // [kt_begin, kt_end) of the one tile that its cluster shares.
     const int splits = SPLITK ? p.splits : 1;
@@ -211,7 +212,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             bool ok = true;
             for (int tile = tile_first; ok && tile < num_tiles; tile += tile_step) {
                 int m_blk, n_blk;
-                tile_coords(p, tile, m_blk, n_blk);
+                tile_coords(p, p.tile_base + tile, m_blk, n_blk);
                 const int sfb_tiles = (2 * n_blk + 1 < p.sf_row_tiles_b) ? 2 : 1;
                 for (int kt = kt_begin; kt < kt_end; ++kt) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status,
@@ -326,7 +327,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         bool ok = true;
         for (int tile = tile_first; ok && tile < num_tiles; tile += tile_step, ++it) {
             int m_blk, n_blk;
-            tile_coords(p, tile, m_blk, n_blk);
+            tile_coords(p, p.tile_base + tile, m_blk, n_blk);
             const int b = it & 1;
             const uint32_t use = (uint32_t)(it >> 1);
             // The bias of this warp's 128 columns goes to shared memory before the
@@ -503,7 +504,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         cluster_sync_all();
         if (warp >= 2) {
             int m_blk, n_blk;
-            tile_coords(p, tile_first, m_blk, n_blk);
+            tile_coords(p, p.tile_base + tile_first, m_blk, n_blk);
             const int rows = min(BM, p.M - m_blk * BM);
             const int r_lo = rank * rows / splits, r_hi = (rank + 1) * rows / splits;
             const uint32_t part = smem_u32(smem);
@@ -706,6 +707,8 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
     p.tma_store = tma_store ? 1 : 0;
     p.n_fast = (N <= M) ? 1 : 0;
     p.splits = 1;
+    p.tile_base = 0;
+    p.tile_count = p.m_blocks * p.n_blocks;
     if (QOUT) {
         p.q_packed = q->packed;
         p.q_sf = q->sf;
@@ -721,6 +724,27 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
         if (splits > 1) {
             p.splits = splits;
             return launch_split_k(mapA, mapB, mapY, p, tiles * splits, splits, stream);
+        }
+        // One full wave plus a short second one (at most SMs / 2 tiles) of long tiles
+        // (K >= 4096): the full wave runs persistent, the leftover tiles split K over
+        // clusters right behind it (1024 x 5120 x 5120: 148 + 12 tiles, 37.1 -> 34.1 us
+        // on B200).  A split-K launch costs about 15 us of fixed time, so it loses where
+        // it replaces only the last of many waves or a short-K wave.
+        const int tail = tiles % dev.sms;
+        if (tiles > dev.sms && tiles < 2 * dev.sms && tail > 0 && p.k_tiles >= 16) {
+            const int ts = choose_splits(tail, p.k_tiles, dev);
+            if (ts > 1) {
+                GemmParams full = p;
+                full.tile_count = tiles - tail;
+                if (launch_pdl(gemm_kernel<false, false, false>, (unsigned)dev.sms, THREADS,
+                               SMEM_BYTES, stream, mapA, mapB, mapY, full) != cudaSuccess)
+                    return NVFP4_ERR_CUDA;
+                GemmParams rest = p;
+                rest.tile_base = tiles - tail;
+                rest.tile_count = tail;
+                rest.splits = ts;
+                return launch_split_k(mapA, mapB, mapY, rest, tail * ts, ts, stream);
+            }
         }
     }
     const int grid = tiles < dev.sms ? tiles : dev.sms;

@@ -68,18 +68,24 @@ def test_gemm_parity(oracle, M, N, K, bias):
     run_gemm_case(oracle, M, N, K, bias, seed=M * 31 + N * 7 + K)
 
 
-@pytest.mark.parametrize("M,N,K,rows", [
-    (16, 5120, 5120, None),      # the M-sweep's decode shapes: 20 tiles on 148 SMs
-    (128, 5120, 5120, 24),
-    (7, 2050, 768, None),        # N % 4 != 0: element-wise stores of the reduced rows
-    (1, 64, 4096, None),
-    (130, 520, 1536, None),      # two row blocks, ragged N and M
+@pytest.mark.parametrize("M,N,K,rows,cols", [
+    (16, 5120, 5120, None, None),     # the M-sweep's decode shapes: 20 tiles on 148 SMs
+    (128, 5120, 5120, 24, None),
+    (7, 2050, 768, None, None),       # N % 4 != 0: element-wise stores of the reduced rows
+    (1, 64, 4096, None, None),
+    (130, 520, 1536, None, None),     # two row blocks, ragged N and M
+    # one full wave plus a short second one of long tiles: the full wave runs
+    # persistent, the leftover tiles split K (160 = 148 + 12 and 162 = 148 + 14 tiles)
+    (1024, 5120, 5120, 192, 192),
+    (1152, 4608, 4096, 128, 128),
 ])
-def test_gemm_split_k(oracle, M, N, K, rows):
+def test_gemm_split_k(oracle, M, N, K, rows, cols):
     """Grids with at most half as many tiles as SMs split K over a cluster of CTAs and
-    reduce the partial tiles over distributed shared memory."""
+    reduce the partial tiles over distributed shared memory; so does the short last
+    wave of a larger grid."""
     sel = None if rows is None else sample_rows(M, rows, seed=M + N)
-    run_gemm_case(oracle, M, N, K, bias=True, seed=M * 13 + N + K, rows=sel)
+    csel = None if cols is None else sample_rows(N, cols, seed=N + K)
+    run_gemm_case(oracle, M, N, K, bias=True, seed=M * 13 + N + K, rows=sel, cols=csel)
 
 
 def test_gemm_split_k_deterministic_and_graph_capturable():
