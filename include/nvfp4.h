@@ -25,7 +25,11 @@
  *     synchronises (except nvfp4_last_device_status, which says so); each call only
  *     enqueues kernels on `stream` (a cudaStream_t; NULL = legacy default stream),
  *     so calls are stream-ordered and may be captured in a CUDA graph
- *     (nvfp4_linear_fixed_scratch states its own set-up condition).
+ *     (nvfp4_linear_fixed_scratch states its own set-up condition).  The quantizer
+ *     and GEMM kernels are launched with programmatic stream serialization: their
+ *     set-up (barriers, tensor memory) may overlap the end of the previous kernel on
+ *     the stream, but they wait for it to complete before touching any global
+ *     memory, so the stream order holds for every input and output.
  *   - bf16 tensors are row-major with no padding; tensor pointers must be 16-byte
  *     aligned, scalar pointers 4-byte aligned.
  *   - Argument checks run on the host before anything is enqueued; on any error
