@@ -6,15 +6,18 @@ tiles of 4096 tokens batched -- qkv [3072,1024], attn-out [1024,1024], FFN-in
 [4096,1024], FFN-out [1024,4096], M = 32768 -- each with a 128-wide block Hadamard
 folded into the weight, the dynamic activation scale (per-call amax), bias, bf16
 output.  Per linear the step runs the whole path: rotate + amax pass, rotate +
-quantize pass (nvfp4_quantize) and the block-scaled GEMM (nvfp4_gemm), exactly the
-launches nvfp4_linear makes, with CUDA events between them so the quantizer and the
-GEMM are timed separately on the launching stream.  Inputs are seeded synthetic
-tensors already in HBM; the activations of one step (448 MiB) exceed the 126 MB L2.
+quantize pass (nvfp4_quantize) and the block-scaled GEMM (nvfp4_gemm_prepared, the
+weight scales prepared offline with the packing), exactly the launches
+nvfp4_linear_prepared makes.  The K timed steps run back to back; a second pass with
+CUDA events between the launches times the quantizer and the GEMM separately.  Inputs
+are seeded synthetic tensors already in HBM; the activations of one step (448 MiB)
+exceed the 126 MB L2.
 
 Also measured in the same run: the static-scale variant of the step, offline weight
-packing (hadamard_rotate + nvfp4_quantize on the four weights), and the end-to-end
-path through nvfp4_linear with pinned host buffers (H2D of x and D2H of y inside the
-timed region).  The CPU baseline is the oracle on a bounded row sample.
+packing of one Qwen3-VL text-encoder layer, NVFP4 -> bf16 expansion, the fused FFN
+pair, the int8 W8A8 block, a GEMM M-sweep at N = K = 5120, and the end-to-end path
+through nvfp4_linear_prepared with pinned host buffers (H2D of x and D2H of y inside
+the timed region).  The CPU baseline is the oracle on a bounded row sample.
 
 Prints one JSON line (rank 0).  --impl reference times the oracle instead.
 Multi-GPU (torchrun): every rank runs its own independent batch (weak scaling, no
@@ -46,8 +49,8 @@ METRIC = "nvfp4_linear TFLOPS (% of dense FP4 peak); quantizer GB/s (% of HBM)"
 # profiles/vit_block_step_launches.md, valid only for the kernel sources it was taken on
 # (sha256 prefix); reported as null once a source has changed.
 MEASURED_TRAFFIC = {
-    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "4627cccceb79e122",
-             "bytes_per_step": 529.5e6},
+    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "385bfdc4d0e367d2",
+             "bytes_per_step": 533.3e6},
     "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "6de0f6e3f8099c0b",
               "bytes_per_step": 959.1e6},
 }
@@ -153,6 +156,8 @@ class Layer:
         self.x = lin.x
         self.bias = lin.bias
         self.wp, self.wsf, self.gsf_w = nv.pack_weight(lin.weight, GROUP)
+        # offline, with the packing: the weight scales in the order the GEMM copies them
+        self.wsf_prep = nv.prepare_weight_scales(self.wsf, self.N, self.K)
         self.xp = torch.empty(self.M, self.K // 2, dtype=torch.uint8, device=dev)
         self.xsf = torch.empty(nv.nvfp4_scale_bytes(self.M, self.K), dtype=torch.uint8, device=dev)
         self.scalars = torch.empty(2, dtype=torch.float32, device=dev)
@@ -173,8 +178,9 @@ class Layer:
 
 def run_step(layers, dynamic: bool, events=None):
     """One pass of the path over the four linears -- the same two entry points and three
-    launches per linear that nvfp4_linear makes (amax + quantize writing alpha, then the
-    GEMM); events[i] = (e0, e1, e2) per linear bracket the quantizer and the GEMM."""
+    launches per linear that nvfp4_linear_prepared makes (amax + quantize writing alpha,
+    then the GEMM); events[i] = (e0, e1, e2) per linear bracket the quantizer and the
+    GEMM."""
     L = nv.lib()
     s = nv._stream()
     for i, ly in enumerate(layers):
@@ -189,11 +195,11 @@ def run_step(layers, dynamic: bool, events=None):
             raise nv.NVFP4Error("nvfp4_quantize", st)
         if events is not None:
             events[i][1].record()
-        st = L.nvfp4_gemm(nv._ptr(ly.xp), nv._ptr(ly.xsf), nv._ptr(ly.wp), nv._ptr(ly.wsf),
-                          nv._ptr(ly.scalars[1:]), nv._ptr(ly.bias), nv._ptr(ly.y), ly.M, ly.N,
-                          ly.K, s)
+        st = L.nvfp4_gemm_prepared(nv._ptr(ly.xp), nv._ptr(ly.xsf), nv._ptr(ly.wp),
+                                   nv._ptr(ly.wsf_prep), nv._ptr(ly.scalars[1:]),
+                                   nv._ptr(ly.bias), nv._ptr(ly.y), ly.M, ly.N, ly.K, s)
         if st:
-            raise nv.NVFP4Error("nvfp4_gemm", st)
+            raise nv.NVFP4Error("nvfp4_gemm_prepared", st)
         if events is not None:
             events[i][2].record()
 
@@ -251,7 +257,7 @@ def rank_seed(rank: int) -> int:
 
 
 def e2e_steps(layers, steps, warmup, dist_on):
-    """Through the public nvfp4_linear call with pinned host buffers: per step, H2D of
+    """Through the public nvfp4_linear_prepared call with pinned host buffers: per step, H2D of
     every linear's x, the linear, D2H of every y (all on the current stream)."""
     host_x = [ly.x.cpu().pin_memory() for ly in layers]
     host_y = [torch.empty(ly.y.shape, dtype=torch.bfloat16).pin_memory() for ly in layers]
@@ -260,8 +266,8 @@ def e2e_steps(layers, steps, warmup, dist_on):
     def step():
         for i, ly in enumerate(layers):
             dev_x[i].copy_(host_x[i], non_blocking=True)
-            nv.nvfp4_linear(dev_x[i], ly.wp, ly.wsf, ly.gsf_w, ly.N, bias=ly.bias,
-                            rotate_group=GROUP, workspace=ly.lin_ws, out=ly.y)
+            nv.nvfp4_linear(dev_x[i], ly.wp, ly.wsf_prep, ly.gsf_w, ly.N, bias=ly.bias,
+                            rotate_group=GROUP, workspace=ly.lin_ws, out=ly.y, prepared=True)
             host_y[i].copy_(ly.y, non_blocking=True)
 
     for _ in range(warmup):
@@ -498,6 +504,7 @@ def m_sweep(dev, pk):
         return packed, sf
 
     wp, wsf = operand(N)
+    wsf = nv.prepare_weight_scales(wsf, N, K)
     alpha = torch.tensor([1e-3], device=dev)
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
     points = []
@@ -505,13 +512,13 @@ def m_sweep(dev, pk):
         xp, xsf = operand(M)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         for _ in range(3):
-            nv.nvfp4_gemm(xp, xsf, wp, wsf, alpha, None, M, N, K, out=y)
+            nv.nvfp4_gemm_prepared(xp, xsf, wp, wsf, alpha, None, M, N, K, out=y)
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(10)]
         for e0, e1 in evs:
             flush.fill_(1.0)
             e0.record()
-            nv.nvfp4_gemm(xp, xsf, wp, wsf, alpha, None, M, N, K, out=y)
+            nv.nvfp4_gemm_prepared(xp, xsf, wp, wsf, alpha, None, M, N, K, out=y)
             e1.record()
         torch.cuda.synchronize()
         ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / len(evs)
@@ -522,7 +529,8 @@ def m_sweep(dev, pk):
                        "frac_of_hbm": gb / pk["hbm"]})
         del xp, xsf, y
     del flush
-    return {"workload": "nvfp4_gemm, N = K = 5120, no bias, L2 flushed before each launch",
+    return {"workload": "nvfp4_gemm_prepared, N = K = 5120, no bias, L2 flushed before each "
+                        "launch",
             "points": points}
 
 
@@ -612,7 +620,7 @@ def run_ours(args, dist_on, rank, world, local_rank):
     dominant_is_gemm = g_time >= q_time
     gemm_roof = {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                  "frac": gemm_tflops / fp4_peak, "traffic": measured_traffic("gemm"),
-                 "traffic_unit": "bytes per step (4 launches)", "kernel": "gemm_kernel",
+                 "traffic_unit": "bytes per step (4 launches)", "kernel": "gemm_kernel (prepared weight scales)",
                  "per_linear_ms": g_ms, "algorithmic_flop": flops,
                  "frac_of_nominal_9PF": gemm_tflops / 9000.0,
                  "peak_note": f"{pk['src']}: 4 x bf16 sustained ({pk['bf16_sus']} TFLOP/s), "
@@ -652,7 +660,7 @@ def run_ours(args, dist_on, rank, world, local_rank):
         "m_sweep": msweep,
         "e2e": {"value": aggregate_tflops(flops, e2e_ms, world), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": "nvfp4_linear"},
+                "api": "nvfp4_linear_prepared"},
         "gpu_launches": 3 * len(layers) * args.steps,
         "clocks": clk,
     }

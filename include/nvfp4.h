@@ -159,6 +159,34 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const ui
                         void* y_bf16, int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
+ * nvfp4_prepare_weight_scales -- a weight's 128x4 block scales rearranged once, offline,
+ * for nvfp4_gemm_prepared / nvfp4_linear_prepared (same page and operation as
+ * nvfp4_gemm; only the order of the B scale bytes differs).  For each 256-row block nb of
+ * W and each K step k of 64 values there is one 4 KiB slot, at (nb * K/64 + k) * 4096;
+ * inside it, for row group g = 0..15 and half h = 0, 1, the 128 bytes at g*256 + h*128
+ * are bytes (g % 4) * 128 .. +127 of the 512-byte 128x4 chunk of row tile 2*nb + h and
+ * step k (zero where that row tile is past N).  That is the shared-memory source of one
+ * tcgen05.cp 128x256b per K step for both 128-row halves of a B tile, which fills the
+ * same tensor-memory columns as two 32x128b.warpx4 copies of the 128x4 chunks.
+ *   sf  : in,  the weight's 128x4 scales (nvfp4_scale_bytes(N, K) bytes)
+ *   out : out, nvfp4_prepared_scale_bytes(N, K) bytes, caller-owned
+ *   K % 64 == 0.  Errors: INVALID_ARG, SHAPE, ALIGN (16-byte), DEVICE, CUDA.
+ */
+NVFP4_API size_t nvfp4_prepared_scale_bytes(int64_t N, int64_t K);
+NVFP4_API nvfp4_status nvfp4_prepare_weight_scales(const uint8_t* sf, int64_t N, int64_t K,
+                                                   uint8_t* out, void* stream);
+
+/*
+ * nvfp4_gemm_prepared -- nvfp4_gemm with the weight scales from
+ * nvfp4_prepare_weight_scales (sfb_prepared); arguments, result (bit for bit) and errors
+ * otherwise as nvfp4_gemm.  Two tensor-memory scale copies per K step instead of three.
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_prepared(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                           const uint8_t* sfb_prepared, const float* alpha,
+                                           const void* bias_bf16, void* y_bf16, int64_t M,
+                                           int64_t N, int64_t K, void* stream);
+
+/*
  * nvfp4_gemm_quantize_out -- nvfp4_gemm whose epilogue hands the next linear its NVFP4
  * input directly: the bf16 product y = bf16(alpha * acc + bias) is encoded in
  * registers under a static global scale and only the codes and scales are written
@@ -207,6 +235,19 @@ NVFP4_API nvfp4_status nvfp4_linear(const void* x_bf16, int64_t M, int64_t K, co
                           const uint8_t* w_sf, const float* gsf_w, int64_t N,
                           const void* bias_bf16, const float* gsf_x, int rotate_group,
                           void* workspace, size_t ws_bytes, void* y_bf16, void* stream);
+
+/*
+ * nvfp4_linear_prepared -- nvfp4_linear with the weight scales from
+ * nvfp4_prepare_weight_scales (w_sf_prepared); arguments, workspace, result (bit for bit)
+ * and errors otherwise as nvfp4_linear.
+ */
+NVFP4_API nvfp4_status nvfp4_linear_prepared(const void* x_bf16, int64_t M, int64_t K,
+                                             const uint8_t* w_packed,
+                                             const uint8_t* w_sf_prepared, const float* gsf_w,
+                                             int64_t N, const void* bias_bf16,
+                                             const float* gsf_x, int rotate_group,
+                                             void* workspace, size_t ws_bytes, void* y_bf16,
+                                             void* stream);
 
 /*
  * nvfp4_dequantize -- NVFP4 -> bf16 expansion of a packed tensor, the W4A16 path for

@@ -35,6 +35,9 @@ SIGNATURES = {
     "nvfp4_quantize": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                               _vp]),
     "nvfp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "nvfp4_gemm_prepared": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+    "nvfp4_prepared_scale_bytes": (_sz, [_i64, _i64]),
+    "nvfp4_prepare_weight_scales": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "nvfp4_dequantize": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
     "int8_quantize_rows": (_int, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "int8_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp]),
@@ -45,6 +48,8 @@ SIGNATURES = {
     "nvfp4_linear_workspace_bytes": (_sz, [_i64, _i64]),
     "nvfp4_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _int, _vp, _sz, _vp,
                             _vp]),
+    "nvfp4_linear_prepared": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _int, _vp,
+                                     _sz, _vp, _vp]),
     "nvfp4_linear_fixed_scratch": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _int,
                                           _vp, _vp]),
     "nvfp4_last_device_status": (_int, [_vp, ctypes.POINTER(_int)]),
@@ -180,12 +185,42 @@ def nvfp4_gemm(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.T
     return y
 
 
+def nvfp4_prepared_scale_bytes(N: int, K: int) -> int:
+    return lib().nvfp4_prepared_scale_bytes(N, K)
+
+
+def prepare_weight_scales(sf: torch.Tensor, N: int, K: int, out: torch.Tensor | None = None,
+                          stream=None) -> torch.Tensor:
+    """A weight's 128x4 scales in the order nvfp4_gemm_prepared / nvfp4_linear_prepared
+    read (one 4 KiB slot per 256-row block and K step)."""
+    if out is None:
+        out = torch.empty(max(nvfp4_prepared_scale_bytes(N, K), 1), dtype=torch.uint8,
+                          device=sf.device)
+    _check("nvfp4_prepare_weight_scales",
+           lib().nvfp4_prepare_weight_scales(_ptr(sf), N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def nvfp4_gemm_prepared(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,
+                        sfb_prepared: torch.Tensor, alpha: torch.Tensor,
+                        bias: torch.Tensor | None, M: int, N: int, K: int,
+                        out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """nvfp4_gemm with the weight scales from prepare_weight_scales."""
+    alpha = _scalar(alpha, a.device, "alpha")
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=a.device) if out is None else out
+    _check("nvfp4_gemm_prepared", lib().nvfp4_gemm_prepared(
+        _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb_prepared), _ptr(alpha), _ptr(bias), _ptr(y), M, N,
+        K, _stream(stream)))
+    return y
+
+
 def nvfp4_linear(x: torch.Tensor, w_packed: torch.Tensor, w_sf: torch.Tensor,
                  gsf_w: torch.Tensor, N: int, bias: torch.Tensor | None = None,
                  gsf_x: torch.Tensor | float | None = None, rotate_group: int = 0,
                  workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
-                 stream=None) -> torch.Tensor:
-    """The whole W4A4 linear: bf16 x [M, K] with a packed weight [N, K/2] -> bf16 [M, N]."""
+                 stream=None, prepared: bool = False) -> torch.Tensor:
+    """The whole W4A4 linear: bf16 x [M, K] with a packed weight [N, K/2] -> bf16 [M, N].
+    With prepared=True, w_sf is the output of prepare_weight_scales."""
     _bf16_2d(x, "x")
     M, K = x.shape
     gsf_x = _scalar(gsf_x, x.device, "gsf_x")
@@ -194,7 +229,8 @@ def nvfp4_linear(x: torch.Tensor, w_packed: torch.Tensor, w_sf: torch.Tensor,
         workspace = torch.empty(nvfp4_linear_workspace_bytes(M, K), dtype=torch.uint8,
                                 device=x.device)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
-    _check("nvfp4_linear", lib().nvfp4_linear(
+    name = "nvfp4_linear_prepared" if prepared else "nvfp4_linear"
+    _check(name, getattr(lib(), name)(
         _ptr(x), M, K, _ptr(w_packed), _ptr(w_sf), _ptr(gsf_w), N, _ptr(bias), _ptr(gsf_x),
         int(rotate_group), _ptr(workspace), workspace.numel(), _ptr(y), _stream(stream)))
     return y

@@ -206,6 +206,41 @@ nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
     return launch_gemm(a, sfa, b, sfb, alpha, bias, y, M, N, K, static_cast<cudaStream_t>(stream));
 }
 
+nvfp4_status nvfp4_gemm_prepared(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                 const uint8_t* sfb_prepared, const float* alpha, const void* bias,
+                                 void* y, int64_t M, int64_t N, int64_t K, void* stream) {
+    if (!a || !sfa || !b || !sfb_prepared || !alpha || !y || M < 0 || N < 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 64 || K >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+    if (!aligned(a, 16) || !aligned(sfa, 16) || !aligned(b, 16) || !aligned(sfb_prepared, 16) ||
+        !aligned(y, 16) || !aligned(alpha, 4) || (bias && !aligned(bias, 16)))
+        return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    return launch_gemm_prepared(a, sfa, b, sfb_prepared, alpha, bias, y, M, N, K,
+                                static_cast<cudaStream_t>(stream));
+}
+
+size_t nvfp4_prepared_scale_bytes(int64_t N, int64_t K) {
+    if (N < 0 || K <= 0 || K % 64 || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return 0;
+    return prepared_scale_bytes(N, K);
+}
+
+nvfp4_status nvfp4_prepare_weight_scales(const uint8_t* sf, int64_t N, int64_t K, uint8_t* out,
+                                         void* stream) {
+    if (!sf || !out || N < 0 || N >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 64 || K >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+    if (!aligned(sf, 16) || !aligned(out, 16)) return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (N == 0) return NVFP4_OK;
+    return launch_prepare_scales(sf, N, K, out, static_cast<cudaStream_t>(stream));
+}
+
 nvfp4_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* sf, const float* gsf,
                               int64_t rows, int64_t K, void* y, void* stream) {
     if (!packed || !sf || !gsf || !y || rows < 0) return NVFP4_ERR_INVALID_ARG;
@@ -302,10 +337,12 @@ size_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K) {
     return linear_ws(M, K).total;
 }
 
-nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w_packed,
-                          const uint8_t* w_sf, const float* gsf_w, int64_t N, const void* bias,
-                          const float* gsf_x, int group, void* workspace, size_t ws_bytes,
-                          void* y, void* stream) {
+// nvfp4_linear and nvfp4_linear_prepared: the same checks and launches; `prepared` says
+// which order w_sf is in (128x4, or nvfp4_prepare_weight_scales).
+static nvfp4_status linear_impl(const void* x, int64_t M, int64_t K, const uint8_t* w_packed,
+                         const uint8_t* w_sf, const float* gsf_w, int64_t N, const void* bias,
+                         const float* gsf_x, int group, void* workspace, size_t ws_bytes,
+                         void* y, void* stream, bool prepared) {
     if (!x || !w_packed || !w_sf || !gsf_w || !y || M < 0 || N < 0 || !valid_group(group))
         return NVFP4_ERR_INVALID_ARG;
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARG;
@@ -331,7 +368,25 @@ nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w_
     st = launch_quantize(x, M, K, group, gsf_x, &scalars[0], xp, xsf, partials, gsf_w, &scalars[1],
                          s);
     if (st != NVFP4_OK) return st;
+    if (prepared)
+        return launch_gemm_prepared(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s);
     return launch_gemm(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s);
+}
+
+nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w_packed,
+                          const uint8_t* w_sf, const float* gsf_w, int64_t N, const void* bias,
+                          const float* gsf_x, int group, void* workspace, size_t ws_bytes,
+                          void* y, void* stream) {
+    return linear_impl(x, M, K, w_packed, w_sf, gsf_w, N, bias, gsf_x, group, workspace,
+                       ws_bytes, y, stream, false);
+}
+
+nvfp4_status nvfp4_linear_prepared(const void* x, int64_t M, int64_t K, const uint8_t* w_packed,
+                                   const uint8_t* w_sf_prepared, const float* gsf_w, int64_t N,
+                                   const void* bias, const float* gsf_x, int group,
+                                   void* workspace, size_t ws_bytes, void* y, void* stream) {
+    return linear_impl(x, M, K, w_packed, w_sf_prepared, gsf_w, N, bias, gsf_x, group, workspace,
+                       ws_bytes, y, stream, true);
 }
 
 nvfp4_status nvfp4_linear_fixed_scratch(const void* x, int64_t M, int64_t K,

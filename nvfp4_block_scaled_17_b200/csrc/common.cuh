@@ -431,6 +431,21 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t smem_addr) {
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// 128 lanes x 256 bits (8 columns) from shared memory, lane l from source row l.
+__device__ __forceinline__ void tc_copy_sf_128x256(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
+// Descriptor for tcgen05.cp of a 128-row x 32-byte block stored as 8-row x 16-byte core
+// matrices, core matrix (g, h) (row group g, 16-byte half h) at g * 256 + h * 128: no
+// swizzle, leading-dimension offset 128, stride offset 256.  Read either way round the
+// two offsets stay inside the 4 KiB block.
+__device__ __forceinline__ uint64_t sdesc_sf_rep(uint32_t smem_addr) {
+    return (uint64_t)((smem_addr >> 4) & 0x3fffu) | ((uint64_t)(128 >> 4) << 16) |
+           ((uint64_t)(256 >> 4) << 32) | ((uint64_t)1 << 46);
+}
+
 // Descriptor for tcgen05.cp of a 32-row x 16-byte block: no swizzle, 8-row core
 // matrices 128 bytes apart.
 __device__ __forceinline__ uint64_t sdesc_sf(uint32_t smem_addr) {

@@ -58,12 +58,22 @@ constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int SMEM_A = BM * BKB;        // 16 KiB
 constexpr int SMEM_B = BN * BKB;        // 32 KiB
 constexpr int SMEM_SFA = 4 * 512;       // four K=64 scale chunks for 128 rows
-constexpr int SMEM_SFB = 8 * 512;       // the same for 256 rows (two 128-row tiles)
 constexpr int STG_BYTES = 32 * 64;      // one 32 x 32 bf16 staging tile
-constexpr int SMEM_STG = EPI_WARPS * 2 * STG_BYTES;
 constexpr int SMEM_BIAS = EPI_WARPS * 256;   // each epilogue warp's 128 bias values of a tile
-constexpr int SMEM_BYTES =
-    1024 + STAGES * (SMEM_A + SMEM_B + SMEM_SFA + SMEM_SFB) + SMEM_STG + SMEM_BIAS + 256;
+// Shared memory of one build.  B scales per stage: four 512-byte chunks per 128-row half
+// in the 128x4 layout; or (RSB, prepared weight scales) one 4 KiB slot per K step, both
+// halves replicated for a single 128x256b copy, which leaves room for one staging tile
+// per epilogue warp instead of two.
+template <bool RSB>
+struct GemmSmem {
+    static constexpr int SFB = RSB ? 4 * 4096 : 8 * 512;
+    static constexpr int STG_BUFS = RSB ? 1 : 2;
+    static constexpr int STG = EPI_WARPS * STG_BUFS * STG_BYTES;
+    static constexpr int BYTES =
+        1024 + STAGES * (SMEM_A + SMEM_B + SMEM_SFA + SFB) + STG + SMEM_BIAS + 256;
+};
+static_assert(GemmSmem<false>::BYTES <= 232448 && GemmSmem<true>::BYTES <= 232448,
+              "dynamic shared memory above the 227 KiB a CTA can have");
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t TMEM_BUF1 = 192;     // second accumulator buffer (overlaps [192, 256))
 constexpr uint32_t TMEM_SF = 448;       // ring of scale-factor slots
@@ -145,19 +155,20 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& 
     }
 }
 
-template <bool QOUT, bool I8, bool SPLITK>
+template <bool QOUT, bool I8, bool SPLITK, bool RSB>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
+    using SM = GemmSmem<RSB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + STAGES * SMEM_A;
     uint8_t* sStg = sB + STAGES * SMEM_B;
-    uint8_t* sSFA = sStg + SMEM_STG;
+    uint8_t* sSFA = sStg + SM::STG;
     uint8_t* sSFB = sSFA + STAGES * SMEM_SFA;
-    uint8_t* sBias = sSFB + STAGES * SMEM_SFB;
+    uint8_t* sBias = sSFB + STAGES * SM::SFB;
     uint64_t* full = reinterpret_cast<uint64_t*>(sBias + SMEM_BIAS);
     uint64_t* empty = full + STAGES;
     uint64_t* acc_full = empty + STAGES;     // [2]
@@ -222,17 +233,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     }
                     const int steps = min(4, p.kchunks - 4 * kt);
                     const uint32_t sf_bytes = I8 ? 0u : (uint32_t)steps * 512u;
-                    mbar_arrive_expect_tx(&full[stage], SMEM_A + SMEM_B + sf_bytes * (1 + sfb_tiles));
+                    // B scales: per 128-row half, or (RSB) one 4 KiB prepared slot per step
+                    const uint32_t sfb_bytes = RSB ? (uint32_t)steps * 4096u : sf_bytes * sfb_tiles;
+                    mbar_arrive_expect_tx(&full[stage], SMEM_A + SMEM_B + sf_bytes + sfb_bytes);
                     tma_load_2d(sA + stage * SMEM_A, &tmA, &full[stage], kt * BKB, m_blk * BM);
                     tma_load_2d(sB + stage * SMEM_B, &tmB, &full[stage], kt * BKB, n_blk * BN);
                     if constexpr (!I8) {
                         bulk_load(sSFA + stage * SMEM_SFA,
                                   p.sfa + ((size_t)m_blk * p.kchunks + 4 * kt) * 512, sf_bytes,
                                   &full[stage]);
-                        for (int t = 0; t < sfb_tiles; ++t)
-                            bulk_load(sSFB + stage * SMEM_SFB + t * 2048,
-                                      p.sfb + ((size_t)(2 * n_blk + t) * p.kchunks + 4 * kt) * 512,
-                                      sf_bytes, &full[stage]);
+                        if constexpr (RSB) {
+                            bulk_load(sSFB + stage * SM::SFB,
+                                      p.sfb + ((size_t)n_blk * p.kchunks + 4 * kt) * 4096,
+                                      sfb_bytes, &full[stage]);
+                        } else {
+                            for (int t = 0; t < sfb_tiles; ++t)
+                                bulk_load(sSFB + stage * SM::SFB + t * 2048,
+                                          p.sfb + ((size_t)(2 * n_blk + t) * p.kchunks + 4 * kt) * 512,
+                                          sf_bytes, &full[stage]);
+                        }
                     }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -281,7 +300,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     const uint32_t a0 = smem_u32(sA + stage * SMEM_A);
                     const uint32_t b0 = smem_u32(sB + stage * SMEM_B);
                     const uint32_t sfa0 = smem_u32(sSFA + stage * SMEM_SFA);
-                    const uint32_t sfb0 = smem_u32(sSFB + stage * SMEM_SFB);
+                    const uint32_t sfb0 = smem_u32(sSFB + stage * SM::SFB);
                     for (int kk = 0; kk < steps; ++kk) {
                         if constexpr (I8) {
                             mma_i8(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
@@ -291,8 +310,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                             const uint32_t sfa_t = tmem + TMEM_SF + 12u * (uint32_t)sf_slot;
                             const uint32_t sfb_t = sfa_t + 4;
                             tc_copy_sf(sfa_t, sdesc_sf(sfa0 + 512 * kk));
-                            tc_copy_sf(sfb_t, sdesc_sf(sfb0 + 512 * kk));
-                            tc_copy_sf(sfb_t + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
+                            if constexpr (RSB) {
+                                // both 128-row halves of the step in one copy: the same
+                                // 8 columns the two warpx4 copies below fill
+                                tc_copy_sf_128x256(sfb_t, sdesc_sf_rep(sfb0 + 4096 * kk));
+                            } else {
+                                tc_copy_sf(sfb_t, sdesc_sf(sfb0 + 512 * kk));
+                                tc_copy_sf(sfb_t + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
+                            }
                             mma_nvf4(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
                                      sdesc_kmajor_sw128(b0 + 32 * kk), IDESC, sfa_t, sfb_t,
                                      kt > kt_begin || kk > 0);
@@ -320,7 +345,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const int half = (warp - 2) >> 2;
         const float alpha = I8 ? 0.0f : *p.alpha;
         const float qgsf = QOUT ? *p.q_gsf : 0.0f;
-        uint8_t* stg = sStg + (warp - 2) * 2 * STG_BYTES;
+        uint8_t* stg = sStg + (warp - 2) * SM::STG_BUFS * STG_BYTES;
         uint32_t* sbias = reinterpret_cast<uint32_t*>(sBias + (warp - 2) * 256);
         int stg_sel = 0;
         int it = 0;
@@ -396,8 +421,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             // the bf16 chunk, staged and stored
             auto store_words = [&](const uint32_t (&packed)[16], int n0) {
                 if (p.tma_store) {
-                    uint8_t* sb = stg + stg_sel * STG_BYTES;
-                    if (lane == 0) bulk_wait_read<1>();   // this buffer's previous store
+                    uint8_t* sb = stg + (SM::STG_BUFS == 2 ? stg_sel * STG_BYTES : 0);
+                    if (lane == 0) {   // this buffer's previous store has read it
+                        if constexpr (SM::STG_BUFS == 2) bulk_wait_read<1>();
+                        else bulk_wait_read<0>();
+                    }
                     __syncwarp();
                     // 64-byte swizzle: 16-byte chunk c of row r sits at c ^ ((r >> 1) & 3)
 #pragma unroll
@@ -590,12 +618,13 @@ struct QuantOut {
 };
 
 // Split-K build: clusters of `splits` CTAs, one tile per cluster.
+template <bool RSB>
 cudaLaunchConfig_t split_k_config(int grid, int splits, cudaStream_t stream,
                                   cudaLaunchAttribute* attr, bool pdl = false) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = GemmSmem<RSB>::BYTES;
     cfg.stream = stream;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)splits;
@@ -608,11 +637,13 @@ cudaLaunchConfig_t split_k_config(int grid, int splits, cudaStream_t stream,
     return cfg;
 }
 
+template <bool RSB>
 bool split_k_attr(int device) {
     static std::atomic<int> done[64];
     if (done[device & 63].load(std::memory_order_acquire)) return true;
-    if (cudaFuncSetAttribute(gemm_kernel<false, false, true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_kernel<false, false, true, RSB>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmSmem<RSB>::BYTES) != cudaSuccess)
         return false;
     done[device & 63].store(1, std::memory_order_release);
     return true;
@@ -621,18 +652,19 @@ bool split_k_attr(int device) {
 // K splits for a grid with too few tiles to fill the SMs: the largest S <= 8 (a portable
 // cluster) with S <= ceil(K / 256) and tiles * S <= SMs whose clusters are all resident
 // at once (cudaOccupancyMaxActiveClusters, cached per device and S); 1 = no split.
+template <bool RSB>
 int choose_splits(int tiles, int k_tiles, const DeviceInfo& dev) {
     if (tiles * 2 > dev.sms || k_tiles < 2) return 1;
-    if (!split_k_attr(dev.device)) return 1;
+    if (!split_k_attr<RSB>(dev.device)) return 1;
     static std::atomic<int> cap[64][9];   // max active clusters + 1 (0 = not queried yet)
     const int smax = min(8, min(k_tiles, dev.sms / tiles));
     for (int sp = smax; sp >= 2; --sp) {
         int c = cap[dev.device & 63][sp].load(std::memory_order_relaxed) - 1;
         if (c < 0) {
             cudaLaunchAttribute attr[2];
-            const cudaLaunchConfig_t cfg = split_k_config(sp * tiles, sp, nullptr, attr);
+            const cudaLaunchConfig_t cfg = split_k_config<RSB>(sp * tiles, sp, nullptr, attr);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<false, false, true>, &cfg) !=
+            if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<false, false, true, RSB>, &cfg) !=
                 cudaSuccess) {
                 (void)cudaGetLastError();
                 n = 0;
@@ -645,21 +677,22 @@ int choose_splits(int tiles, int k_tiles, const DeviceInfo& dev) {
     return 1;
 }
 
+template <bool RSB>
 nvfp4_status launch_split_k(const CUtensorMap& mapA, const CUtensorMap& mapB,
                             const CUtensorMap& mapY, const GemmParams& p, int grid, int splits,
                             cudaStream_t stream) {
     cudaLaunchAttribute attr[2];
-    const cudaLaunchConfig_t cfg = split_k_config(grid, splits, stream, attr, true);
-    if (cudaLaunchKernelEx(&cfg, gemm_kernel<false, false, true>, mapA, mapB, mapY, p) !=
+    const cudaLaunchConfig_t cfg = split_k_config<RSB>(grid, splits, stream, attr, true);
+    if (cudaLaunchKernelEx(&cfg, gemm_kernel<false, false, true, RSB>, mapA, mapB, mapY, p) !=
         cudaSuccess)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
 }
 
-// One launcher for the three builds of the kernel: NVFP4 (sfa/sfb = 128x4 scales,
-// alpha), NVFP4 with the quantized output, and int8 (sfa/sfb unused; sx/sw = fp32 row
-// scales of A and B).
-template <bool QOUT, bool I8>
+// One launcher for the builds of the kernel: NVFP4 (sfa = 128x4 scales; sfb = 128x4
+// scales, or with RSB the prepared weight scales; alpha), NVFP4 with the quantized
+// output, and int8 (sfa/sfb unused; sx/sw = fp32 row scales of A and B).
+template <bool QOUT, bool I8, bool RSB = false>
 nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                               const uint8_t* sfb, const float* alpha, const void* bias, void* y,
                               int64_t M, int64_t N, int64_t K, const QuantOut* q,
@@ -683,8 +716,9 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
 
     static bool attr_set[64] = {false};
     if (!attr_set[dev.device & 63]) {
-        if (cudaFuncSetAttribute(gemm_kernel<QOUT, I8, false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemm_kernel<QOUT, I8, false, RSB>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 GemmSmem<RSB>::BYTES) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         attr_set[dev.device & 63] = true;
     }
@@ -720,10 +754,10 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
 
     const int tiles = p.m_blocks * p.n_blocks;
     if constexpr (!QOUT && !I8) {
-        const int splits = choose_splits(tiles, p.k_tiles, dev);
+        const int splits = choose_splits<RSB>(tiles, p.k_tiles, dev);
         if (splits > 1) {
             p.splits = splits;
-            return launch_split_k(mapA, mapB, mapY, p, tiles * splits, splits, stream);
+            return launch_split_k<RSB>(mapA, mapB, mapY, p, tiles * splits, splits, stream);
         }
         // One full wave plus a short second one (at most SMs / 2 tiles) of long tiles
         // (K >= 4096): the full wave runs persistent, the leftover tiles split K over
@@ -732,35 +766,85 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
         // it replaces only the last of many waves or a short-K wave.
         const int tail = tiles % dev.sms;
         if (tiles > dev.sms && tiles < 2 * dev.sms && tail > 0 && p.k_tiles >= 16) {
-            const int ts = choose_splits(tail, p.k_tiles, dev);
+            const int ts = choose_splits<RSB>(tail, p.k_tiles, dev);
             if (ts > 1) {
                 GemmParams full = p;
                 full.tile_count = tiles - tail;
-                if (launch_pdl(gemm_kernel<false, false, false>, (unsigned)dev.sms, THREADS,
-                               SMEM_BYTES, stream, mapA, mapB, mapY, full) != cudaSuccess)
+                if (launch_pdl(gemm_kernel<false, false, false, RSB>, (unsigned)dev.sms, THREADS,
+                               GemmSmem<RSB>::BYTES, stream, mapA, mapB, mapY, full) != cudaSuccess)
                     return NVFP4_ERR_CUDA;
                 GemmParams rest = p;
                 rest.tile_base = tiles - tail;
                 rest.tile_count = tail;
                 rest.splits = ts;
-                return launch_split_k(mapA, mapB, mapY, rest, tail * ts, ts, stream);
+                return launch_split_k<RSB>(mapA, mapB, mapY, rest, tail * ts, ts, stream);
             }
         }
     }
     const int grid = tiles < dev.sms ? tiles : dev.sms;
-    if (launch_pdl(gemm_kernel<QOUT, I8, false>, (unsigned)grid, THREADS, SMEM_BYTES, stream, mapA,
-                   mapB, mapY, p) != cudaSuccess)
+    if (launch_pdl(gemm_kernel<QOUT, I8, false, RSB>, (unsigned)grid, THREADS,
+                   GemmSmem<RSB>::BYTES, stream, mapA, mapB, mapY, p) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
 }
 
+// Prepared weight scales: the 4 KiB slot of (256-row block nb, K step k) holds, for each
+// 8-row group g (16) and 128-row half h (2), at g * 256 + h * 128, the 128 bytes
+// (g % 4) * 128 .. of the 512-byte 128x4 chunk (row tile 2 nb + h, step k); halves past
+// the last row tile are zero.  One thread per 16 bytes.
+__global__ void __launch_bounds__(256) prepare_scales_kernel(const uint8_t* __restrict__ sf,
+                                                             uint8_t* __restrict__ out,
+                                                             int64_t pieces, int kchunks,
+                                                             int row_tiles) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < pieces;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t slot = i >> 8;
+        const int q = (int)(i & 255);
+        const int g = q >> 4, h = (q >> 3) & 1, part = q & 7;
+        const int64_t nb = slot / kchunks, k = slot - nb * kchunks;
+        const int64_t tile = 2 * nb + h;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (tile < row_tiles)
+            v = *reinterpret_cast<const uint4*>(sf + (tile * kchunks + k) * 512 + (g & 3) * 128 +
+                                                part * 16);
+        *reinterpret_cast<uint4*>(out + slot * 4096 + g * 256 + h * 128 + part * 16) = v;
+    }
+}
+
 }  // namespace
+
+size_t prepared_scale_bytes(int64_t N, int64_t K) {
+    return (size_t)((N + 255) / 256) * (size_t)(K / 64) * 4096u;
+}
+
+nvfp4_status launch_prepare_scales(const uint8_t* sf, int64_t N, int64_t K, uint8_t* out,
+                                   cudaStream_t stream) {
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    const int kchunks = (int)(K / 64);
+    const int64_t pieces = (int64_t)((N + 255) / 256) * kchunks * 256;
+    const int64_t need = (pieces + 255) / 256;
+    const int64_t cap = (int64_t)dev.sms * 8;
+    const int grid = (int)(need < cap ? (need > 0 ? need : 1) : cap);
+    prepare_scales_kernel<<<grid, 256, 0, stream>>>(sf, out, pieces, kchunks,
+                                                    (int)((N + 127) / 128));
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
 
 nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          const uint8_t* sfb, const float* alpha, const void* bias, void* y,
                          int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
     return launch_gemm_impl<false, false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, nullptr,
                                           nullptr, nullptr, stream);
+}
+
+nvfp4_status launch_gemm_prepared(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                  const uint8_t* sfb_prepared, const float* alpha,
+                                  const void* bias, void* y, int64_t M, int64_t N, int64_t K,
+                                  cudaStream_t stream) {
+    return launch_gemm_impl<false, false, true>(a, sfa, b, sfb_prepared, alpha, bias, y, M, N, K,
+                                                nullptr, nullptr, nullptr, stream);
 }
 
 nvfp4_status launch_gemm_quant_out(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,

@@ -54,6 +54,16 @@ nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          const uint8_t* sfb, const float* alpha, const void* bias, void* y,
                          int64_t M, int64_t N, int64_t K, cudaStream_t stream);
 
+// The same GEMM with the weight's scales in the prepared order (launch_prepare_scales):
+// one 128x256b tensor-memory copy per K step for both 128-row halves of a B tile.
+nvfp4_status launch_gemm_prepared(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                  const uint8_t* sfb_prepared, const float* alpha,
+                                  const void* bias, void* y, int64_t M, int64_t N, int64_t K,
+                                  cudaStream_t stream);
+size_t prepared_scale_bytes(int64_t N, int64_t K);
+nvfp4_status launch_prepare_scales(const uint8_t* sf, int64_t N, int64_t K, uint8_t* out,
+                                   cudaStream_t stream);
+
 // The GEMM whose epilogue emits the NVFP4 encoding of its bf16 output instead of the
 // output itself (static global scale gsf_out, 128x4 scales, N % 64 == 0).
 nvfp4_status launch_gemm_quant_out(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,

@@ -54,6 +54,10 @@ def test_sizes_match_oracle(L, oracle):
     ws = L.nvfp4_linear_workspace_bytes(4096, 5120)
     assert ws >= 4096 * 5120 // 2 + oracle.scale_bytes(4096, 5120) + 8
     assert ws % 256 == 0
+    # prepared weight scales: one 4 KiB slot per 256-row block and 64-value K step
+    assert L.nvfp4_prepared_scale_bytes(5120, 5120) == 20 * 80 * 4096
+    assert L.nvfp4_prepared_scale_bytes(300, 576) == 2 * 9 * 4096
+    assert L.nvfp4_prepared_scale_bytes(0, 64) == 0 and L.nvfp4_prepared_scale_bytes(8, 48) == 0
 
 
 def test_quantize_argument_errors(L):
@@ -98,6 +102,18 @@ def test_gemm_and_linear_argument_errors(L):
     h = L.hadamard_rotate
     assert h(A, A, 4, 64, 0, S) == nv.ERR_INVALID_ARG
     assert h(A, A, 4, 96, 64, S) == nv.ERR_SHAPE
+    gp = L.nvfp4_gemm_prepared
+    assert gp(A, A, A, A, A, None, A, 4, 4, 48, S) == nv.ERR_SHAPE            # K % 64
+    assert gp(A, A, A, None, A, None, A, 4, 4, 64, S) == nv.ERR_INVALID_ARG   # no B scales
+    assert gp(A, A, A, MIS, A, None, A, 4, 4, 64, S) == nv.ERR_ALIGN
+    pw = L.nvfp4_prepare_weight_scales
+    assert pw(None, 256, 64, A, S) == nv.ERR_INVALID_ARG
+    assert pw(A, -1, 64, A, S) == nv.ERR_INVALID_ARG
+    assert pw(A, 256, 96, A, S) == nv.ERR_SHAPE
+    assert pw(A, 256, 64, MIS, S) == nv.ERR_ALIGN
+    lp = L.nvfp4_linear_prepared
+    assert lp(A, 4, 64, A, A, A, 8, None, None, 0, A, 16, A, S) == nv.ERR_WORKSPACE
+    assert lp(A, 4, 96, A, A, A, 8, None, None, 0, A, 1 << 20, A, S) == nv.ERR_SHAPE
 
 
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-GPU behaviour")

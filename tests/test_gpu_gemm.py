@@ -195,3 +195,103 @@ def test_probe_error_on_gpu():
     ref = (x.double() @ w.double().T)
     err = float((y.double() - ref).norm() / ref.norm())
     assert abs(err - 0.13) < 0.02, err
+
+
+# ---------------------------------------------------------------------------
+# prepared weight scales (nvfp4_prepare_weight_scales + nvfp4_gemm_prepared)
+# ---------------------------------------------------------------------------
+
+def prepared_layout_np(sf: np.ndarray, N: int, K: int) -> np.ndarray:
+    """The prepared order written out from its definition in the header: per 256-row
+    block nb and K step k a 4 KiB slot; bytes g*256 + h*128 .. +127 of it are bytes
+    (g % 4)*128 .. +127 of the 128x4 chunk (row tile 2 nb + h, step k), zero past N."""
+    kc, tiles, nb = K // 64, (N + 127) // 128, (N + 255) // 256
+    chunks = sf.reshape(-1)[: tiles * kc * 512].reshape(tiles, kc, 4, 128)   # [tile, k, g%4, 128]
+    out = np.zeros((nb, kc, 16, 2, 128), dtype=np.uint8)
+    for h in range(2):
+        t = np.arange(nb) * 2 + h
+        ok = t < tiles
+        out[ok, :, :, h, :] = chunks[t[ok]][:, :, np.arange(16) % 4, :]
+    return out.reshape(-1)
+
+
+def random_operands(M, N, K, seed):
+    g = torch.Generator().manual_seed(seed)
+    ap = torch.randint(0, 256, (M, K // 2), generator=g, dtype=torch.int32).to(torch.uint8)
+    bp = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.int32).to(torch.uint8)
+    sa = (0x30 + torch.randint(0, 16, (nv.nvfp4_scale_bytes(M, K),), generator=g,
+                               dtype=torch.int32)).to(torch.uint8)
+    sb = (0x30 + torch.randint(0, 16, (nv.nvfp4_scale_bytes(N, K),), generator=g,
+                               dtype=torch.int32)).to(torch.uint8)
+    bias = (torch.randn(N, generator=g) * 0.01).to(torch.bfloat16)
+    return ap.to(DEV), sa.to(DEV), bp.to(DEV), sb.to(DEV), bias.to(DEV)
+
+
+@pytest.mark.parametrize("N,K", [(256, 64), (300, 576), (5120, 5120), (1000, 512), (128, 1024)])
+def test_prepare_weight_scales_layout(N, K):
+    g = torch.Generator().manual_seed(N + K)
+    sf = torch.randint(0, 256, (nv.nvfp4_scale_bytes(N, K),), generator=g,
+                       dtype=torch.int32).to(torch.uint8)
+    out = torch.full((nv.nvfp4_prepared_scale_bytes(N, K),), 0xAB, dtype=torch.uint8, device=DEV)
+    nv.prepare_weight_scales(sf.to(DEV), N, K, out=out)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(out), prepared_layout_np(sf.numpy(), N, K))
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (128, 256, 256), (100, 200, 192), (129, 300, 320), (257, 513, 1024), (300, 640, 576),
+    (384, 256, 2048), (16, 5120, 5120), (1024, 5120, 5120), (2048, 3072, 1024), (7, 2050, 768),
+])
+@pytest.mark.parametrize("bias", [True, False])
+def test_gemm_prepared_bit_exact_with_128x4(M, N, K, bias):
+    """Same operands, the weight scales in either order: identical bf16 outputs (the same
+    bytes reach the same tensor-memory columns), through the persistent, split-K and
+    split-last-wave schedules."""
+    ap, sa, bp, sb, b = random_operands(M, N, K, M * 7 + N + K)
+    al = torch.tensor([1e-3], device=DEV)
+    b = b if bias else None
+    y0 = nv.nvfp4_gemm(ap, sa, bp, sb, al, b, M, N, K)
+    y1 = nv.nvfp4_gemm_prepared(ap, sa, bp, nv.prepare_weight_scales(sb, N, K), al, b, M, N, K)
+    torch.cuda.synchronize()
+    assert nv.last_device_status() == nv.OK
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+
+
+def test_gemm_prepared_vit_qkv_full_size(oracle):
+    """ViT qkv projection through the prepared weight scales against the fp64 oracle:
+    256 sampled rows x all columns and all rows x 256 sampled columns."""
+    M, N, K = 32768, 3072, 1024
+    x = W.with_outliers((M, K), 0.01, 20.0, W._gen(21, "cpu"), "cpu")
+    w = W.normal((N, K), 0.02, W._gen(22, "cpu"), "cpu").to(torch.bfloat16)
+    b = W.normal((N,), 0.01, W._gen(23, "cpu"), "cpu").to(torch.bfloat16)
+    xp, xsf, gx = oracle.quantize(W.to_u16(x))
+    wp, wsf, gw = oracle.quantize(W.to_u16(w))
+    al = oracle.alpha(gx, gw)
+    y = nv.nvfp4_gemm_prepared(t(xp), t(xsf), t(wp), nv.prepare_weight_scales(t(wsf), N, K),
+                               torch.tensor([al], device=DEV), b.to(DEV), M, N, K)
+    torch.cuda.synchronize()
+    assert nv.last_device_status() == nv.OK
+    rows = sample_rows(M, 256)
+    y64 = oracle.gemm_f64(xp, xsf, wp, wsf, M, N, K, al, W.to_u16(b), rows=rows)
+    assert_gemm_close(y[torch.from_numpy(rows).to(DEV)], y64, "prepared qkv rows")
+    cols = sample_rows(N, 256, seed=9)
+    yt64 = oracle.gemm_f64(wp, wsf, xp, xsf, N, M, K, al, None, rows=cols)
+    yt64 = yt64 + b.float().numpy().astype(np.float64)[cols][:, None]
+    assert_gemm_close(y[:, torch.from_numpy(cols).to(DEV)].t().contiguous(), yt64,
+                      "prepared qkv columns")
+
+
+@pytest.mark.parametrize("group,dynamic", [(0, True), (128, True), (16, False)])
+def test_linear_prepared_bit_exact(group, dynamic):
+    M, N, K = 200, 384, 512
+    x = W.with_outliers((M, K), 0.005, 30.0, W._gen(31 + group, DEV), DEV)
+    w = W.normal((N, K), 0.02, W._gen(32, DEV), DEV).to(torch.bfloat16)
+    b = W.normal((N,), 0.01, W._gen(33, DEV), DEV).to(torch.bfloat16)
+    wp, wsf, gw = nv.pack_weight(w, group)
+    gx = None if dynamic else 37.5
+    y0 = nv.nvfp4_linear(x, wp, wsf, gw, N, b, gx, group)
+    y1 = nv.nvfp4_linear(x, wp, nv.prepare_weight_scales(wsf, N, K), gw, N, b, gx, group,
+                         prepared=True)
+    torch.cuda.synchronize()
+    assert nv.last_device_status() == nv.OK
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
