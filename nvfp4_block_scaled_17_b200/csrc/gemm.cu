@@ -10,9 +10,14 @@
 //   warp 0      TMA producer: per 256-wide K step, a 128 x 128-byte A box and a
 //               256 x 128-byte B box (128-byte swizzle), plus the matching 512-byte
 //               chunks of the 128x4 scale layout with plain bulk copies (the layout
-//               already is the tensor-memory copy order, so no reshuffle is needed).
+//               already is the tensor-memory copy order, so no reshuffle is needed);
+//               or, for prepared weight scales (RSB), the B scales as one 16 KiB bulk
+//               copy of four 4 KiB per-step slots.
 //   warp 1      MMA issuer (one lane): per K=64 step, tcgen05.cp of the step's scale
-//               chunks into a ring of five tensor-memory slots, then tcgen05.mma
+//               chunks into a ring of five tensor-memory slots -- A and the two B
+//               halves as 32x128b.warpx4, or with RSB A as warpx4 and both B halves as
+//               one 128x256b copy of the step's slot (the same 8 columns; two copies
+//               per step instead of three) -- then tcgen05.mma
 //               kind::mxf4nvf4 block16 (M=128, N=256, K=64), accumulating in tensor
 //               memory; tcgen05.commit releases the stage and, at the end of a tile,
 //               hands the accumulator to the epilogue.  The copy for step g overwrites
@@ -20,7 +25,8 @@
 //               waits for an MMA to stop reading the scales it is about to replace.
 //   warps 2..9  epilogue, two warps per 32-lane tensor-memory quadrant (one per
 //               128-column half): tcgen05.ld, alpha, bias, bf16, a 64-byte-swizzled
-//               shared staging tile, TMA store (bounds clipped by the tensor map).
+//               shared staging tile (two per warp, one with RSB), TMA store (bounds
+//               clipped by the tensor map).
 //
 // Accumulator double buffering within 512 tensor-memory columns: tile buffers
 // occupy columns [0, 256) and [192, 448), the scale-factor ring [448, 508).  The two
@@ -33,7 +39,11 @@
 // same pipeline over its share of the K tiles; the raw fp32 partial tile goes to that
 // CTA's own (now idle) stage buffers, and after a cluster barrier rank r sums its share
 // of the rows over all S partials (distributed shared memory, rank order) and applies
-// alpha and the bias.
+// alpha and the bias.  One full wave plus a short second one of long tiles runs the
+// full wave persistent and splits the leftover tiles that way right behind it.
+//
+// Launches use programmatic stream serialization: set-up overlaps the previous
+// kernel's tail, and griddepcontrol.wait precedes every global access.
 //
 // Every wait is bounded (globaltimer); on expiry the kernel records
 // NVFP4_ERR_TIMEOUT, drains its own copies and MMAs, frees tensor memory and exits.
