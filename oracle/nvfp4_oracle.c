@@ -41,6 +41,7 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define EXPORT __attribute__((visibility("default")))
@@ -323,31 +324,48 @@ EXPORT void ora_dequantize_bf16(const uint8_t* packed, const uint8_t* sf, int64_
 
 /* y[i, n] = alpha * sum_k deq_a(rows[i], k) * deq_b(n, k) + bias[n], in fp64,
  * k ascending; every product is exact in fp64.  rows == NULL means rows 0..M-1
- * (then n_rows = M).  bias_bf16 may be NULL. */
+ * (then n_rows = M).  bias_bf16 may be NULL.  Each operand row is dequantized once
+ * (dequant_elem, exact) and the sum runs over the two dequantized rows; on an
+ * allocation failure every output is NaN. */
 EXPORT void ora_gemm_f64(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          const uint8_t* sfb, int64_t N, int64_t K, float alpha,
                          const uint16_t* bias_bf16, const int64_t* rows, int64_t n_rows,
                          double* y) {
-    int64_t nb = K / 16;
-#pragma omp parallel for schedule(dynamic, 1)
+    double* da = (double*)malloc((size_t)(n_rows > 0 ? n_rows : 1) * (size_t)K * sizeof(double));
+    if (!da) {
+        for (int64_t i = 0; i < n_rows * N; ++i) y[i] = NAN;
+        return;
+    }
+#pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n_rows; ++i) {
         int64_t m = rows ? rows[i] : i;
-        for (int64_t n = 0; n < N; ++n) {
-            double acc = 0.0;
-            for (int64_t j = 0; j < nb; ++j) {
-                double sa = ora_e4m3_decode(sfa[ora_scale_offset(m, j, K)]);
-                double sb = ora_e4m3_decode(sfb[ora_scale_offset(n, j, K)]);
-                for (int64_t k = j * 16; k < j * 16 + 16; ++k) {
-                    uint8_t ba = a[m * (K / 2) + k / 2], bb = b[n * (K / 2) + k / 2];
-                    uint8_t ca = (k & 1) ? (ba >> 4) : (ba & 15);
-                    uint8_t cb = (k & 1) ? (bb >> 4) : (bb & 15);
-                    acc += (ora_e2m1_decode(ca) * sa) * (ora_e2m1_decode(cb) * sb);
-                }
-            }
-            double bias = bias_bf16 ? (double)ora_bf16_to_f32(bias_bf16[n]) : 0.0;
-            y[i * N + n] = (double)alpha * acc + bias;
-        }
+        for (int64_t k = 0; k < K; ++k) da[i * K + k] = dequant_elem(a, sfa, m, k, K);
     }
+    int failed = 0;
+#pragma omp parallel
+    {
+        double* db = (double*)malloc((size_t)K * sizeof(double));
+        if (!db) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 8)
+        for (int64_t n = 0; n < N; ++n) {
+            if (!db) continue;
+            for (int64_t k = 0; k < K; ++k) db[k] = dequant_elem(b, sfb, n, k, K);
+            double bias = bias_bf16 ? (double)ora_bf16_to_f32(bias_bf16[n]) : 0.0;
+            for (int64_t i = 0; i < n_rows; ++i) {
+                const double* ra = da + i * K;
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k) acc += ra[k] * db[k];
+                y[i * N + n] = (double)alpha * acc + bias;
+            }
+        }
+        free(db);
+    }
+    free(da);
+    if (failed)
+        for (int64_t i = 0; i < n_rows * N; ++i) y[i] = NAN;
 }
 
 /* ------------------------------------------------------------------------ */
