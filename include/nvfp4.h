@@ -386,6 +386,25 @@ NVFP4_API nvfp4_status nvfp4_debug_cvt_sweep(uint32_t first, int64_t n, uint8_t*
  */
 NVFP4_API nvfp4_status nvfp4_debug_wait_timeout(int64_t budget_us, void* stream);
 
+/*
+ * nvfp4_debug_gemm_f32 -- nvfp4_gemm (sfb_prepared = 0) or nvfp4_gemm_prepared
+ * (sfb_prepared = 1) built with an unrounded output: the same tile schedule, mainloop
+ * and accumulation order, and the epilogue stores y[m,n] = fp32(alpha * acc) + bias[n]
+ * (fp32 add) instead of rounding it to bf16.  The operation is the one the decoder page
+ * defines ("minimax_h3_nvfp4_decoder" -- nvfp4_linear_inference: mm_fp4 then the bias);
+ * the page's mm_fp4 writes bf16, and the bf16 result of nvfp4_gemm equals this output
+ * rounded to nearest even.  It exists so that the GEMM's accumulation error can be
+ * checked against an fp64 reference without the bf16 output rounding on top.
+ *   a, sfa, b, sfb, alpha, bias_bf16, M, N, K : as nvfp4_gemm / nvfp4_gemm_prepared
+ *   y_f32 : out, fp32 [M, N] row-major, 16-byte aligned, caller-owned
+ * Errors: as nvfp4_gemm; INVALID_ARG also for sfb_prepared other than 0 or 1.
+ */
+NVFP4_API nvfp4_status nvfp4_debug_gemm_f32(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                            const uint8_t* sfb, int sfb_prepared,
+                                            const float* alpha, const void* bias_bf16,
+                                            float* y_f32, int64_t M, int64_t N, int64_t K,
+                                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif

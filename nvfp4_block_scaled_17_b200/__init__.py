@@ -55,6 +55,8 @@ SIGNATURES = {
     "nvfp4_last_device_status": (_int, [_vp, ctypes.POINTER(_int)]),
     "nvfp4_debug_cvt_sweep": (_int, [_u32, _i64, _vp, _vp, _vp, _vp]),
     "nvfp4_debug_wait_timeout": (_int, [_i64, _vp]),
+    "nvfp4_debug_gemm_f32": (_int, [_vp, _vp, _vp, _vp, _int, _vp, _vp, _vp, _i64, _i64, _i64,
+                                    _vp]),
 }
 
 _lib = None
@@ -182,6 +184,20 @@ def nvfp4_gemm(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.T
     y = torch.empty(M, N, dtype=torch.bfloat16, device=a.device) if out is None else out
     _check("nvfp4_gemm", lib().nvfp4_gemm(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(alpha),
                                           _ptr(bias), _ptr(y), M, N, K, _stream(stream)))
+    return y
+
+
+def nvfp4_debug_gemm_f32(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                         alpha: torch.Tensor, bias: torch.Tensor | None, M: int, N: int, K: int,
+                         prepared: bool = False, out: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """The GEMM with its unrounded output: y fp32 [M, N] = fp32(alpha * acc) + bias (the
+    value nvfp4_gemm / nvfp4_gemm_prepared round once to bf16)."""
+    alpha = _scalar(alpha, a.device, "alpha")
+    y = torch.empty(M, N, dtype=torch.float32, device=a.device) if out is None else out
+    _check("nvfp4_debug_gemm_f32", lib().nvfp4_debug_gemm_f32(
+        _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), 1 if prepared else 0, _ptr(alpha), _ptr(bias),
+        _ptr(y), M, N, K, _stream(stream)))
     return y
 
 

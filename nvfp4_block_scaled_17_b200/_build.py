@@ -1,9 +1,9 @@
 """Build step for the CUDA library: nvcc -> an in-tree shared object.
 
 Compiles every ``csrc/*.cu`` for sm_100a only (``-gencode
-arch=compute_100a,code=sm_100a``) with the CUDA runtime linked statically, so the
-library does not depend on the runtime version PyTorch ships.  No GPU is needed
-to build.
+arch=compute_100a,code=sm_100a``), one object per file in parallel under ``_build/``,
+and links them with the CUDA runtime linked statically, so the library does not
+depend on the runtime version PyTorch ships.  No GPU is needed to build.
 """
 from __future__ import annotations
 
@@ -52,14 +52,48 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in inputs())
 
 
+OBJ_DIR = os.path.join(ROOT, "_build")
+
+
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
+    """Each translation unit is compiled to an object in parallel (they share no device
+    symbols), then nvcc links the shared object."""
     if not force and up_to_date():
         return LIB_PATH
-    tmp = LIB_PATH + f".{os.getpid()}.tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *(extra or []), "-o", tmp, *sources()]
+    from concurrent.futures import ThreadPoolExecutor
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    tag = f"{os.getpid()}"
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    jobs = []
+    for src in sources():
+        obj = os.path.join(OBJ_DIR, os.path.basename(src) + f".{tag}.o")
+        cmd = [nvcc(), *compile_flags, "-I", INCLUDE, "-I", CSRC, *(extra or []), "-c", "-o", obj, src]
+        jobs.append((cmd, obj))
     if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
+        for cmd, _ in jobs:
+            print(" ".join(cmd), file=sys.stderr)
+    with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+        results = list(ex.map(lambda j: subprocess.run(j[0], capture_output=True, text=True), jobs))
+    failed = [r for r in results if r.returncode != 0]
+    for r in results:
+        if r.stderr:
+            print(r.stderr, file=sys.stderr, end="")
+    if failed:
+        for _, obj in jobs:
+            if os.path.exists(obj):
+                os.remove(obj)
+        raise RuntimeError("nvcc failed for " + ", ".join(r.args[-1] for r in failed))
+    tmp = LIB_PATH + f".{tag}.tmp"
+    link = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
+            "-Xcompiler", "-fPIC", "-o", tmp, *[obj for _, obj in jobs]]
+    if verbose:
+        print(" ".join(link), file=sys.stderr)
+    try:
+        subprocess.run(link, check=True)
+    finally:
+        for _, obj in jobs:
+            if os.path.exists(obj):
+                os.remove(obj)
     os.replace(tmp, LIB_PATH)
     return LIB_PATH
 

@@ -422,6 +422,26 @@ nvfp4_status nvfp4_linear_fixed_scratch(const void* x, int64_t M, int64_t K,
     return launch_gemm(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s);
 }
 
+nvfp4_status nvfp4_debug_gemm_f32(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                                  const uint8_t* sfb, int sfb_prepared, const float* alpha,
+                                  const void* bias, float* y_f32, int64_t M, int64_t N, int64_t K,
+                                  void* stream) {
+    if (!a || !sfa || !b || !sfb || !alpha || !y_f32 || M < 0 || N < 0 ||
+        (sfb_prepared != 0 && sfb_prepared != 1))
+        return NVFP4_ERR_INVALID_ARG;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return NVFP4_ERR_INVALID_ARG;
+    if (K <= 0 || K % 64 || K >= (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
+    if (!aligned(a, 16) || !aligned(sfa, 16) || !aligned(b, 16) || !aligned(sfb, 16) ||
+        !aligned(y_f32, 16) || !aligned(alpha, 4) || (bias && !aligned(bias, 16)))
+        return NVFP4_ERR_ALIGN;
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return NVFP4_OK;
+    return launch_gemm_f32(a, sfa, b, sfb, sfb_prepared != 0, alpha, bias, y_f32, M, N, K,
+                           static_cast<cudaStream_t>(stream));
+}
+
 nvfp4_status nvfp4_last_device_status(void* stream, int* status) {
     if (!status) return NVFP4_ERR_INVALID_ARG;
     int* dev_ptr = nullptr;

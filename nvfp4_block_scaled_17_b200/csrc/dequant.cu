@@ -12,6 +12,8 @@
 // segment of one row: lane t reads the 4 packed bytes of values 8t..8t+7 (one 128-byte
 // line per warp) and writes their 16 bf16 bytes (one 512-byte run per warp).  A warp's
 // work unit is four consecutive segments of a row, loaded before they are expanded.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -104,16 +106,17 @@ nvfp4_status launch_dequantize(const uint8_t* packed, const uint8_t* sf, const f
     p.upr_div = make_fastdiv(p.upr);
     p.cgroups = (K + 63) / 64;
     // one resident wave: every CTA builds the table once
-    static int per_sm[64] = {0};
-    if (!per_sm[dev.device & 63]) {
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dequant_kernel, kDeqThreads, 0) !=
-                cudaSuccess || n <= 0)
-            n = 4;
-        per_sm[dev.device & 63] = n;
+    static std::atomic<int> per_sm[64];
+    int resident = per_sm[dev.device & 63].load(std::memory_order_relaxed);
+    if (!resident) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, dequant_kernel, kDeqThreads,
+                                                          0) != cudaSuccess ||
+            resident <= 0)
+            resident = 4;
+        per_sm[dev.device & 63].store(resident, std::memory_order_relaxed);
     }
     const int64_t need = ((int64_t)p.total + kDeqThreads / 32 - 1) / (kDeqThreads / 32);
-    const int64_t cap = (int64_t)dev.sms * per_sm[dev.device & 63];
+    const int64_t cap = (int64_t)dev.sms * resident;
     const int grid = (int)(need < cap ? (need > 0 ? need : 1) : cap);
     dequant_kernel<<<grid, kDeqThreads, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;

@@ -103,6 +103,7 @@ struct GemmParams {
     const float* alpha;
     const uint16_t* bias;      // bf16 [N] or null
     uint16_t* y;               // bf16 [M, N]
+    float* y32;                // fp32 [M, N] (the unrounded-output build)
     int M, N;
     int m_blocks, n_blocks;
     int k_tiles;               // ceil(K / 256)
@@ -165,7 +166,7 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& 
     }
 }
 
-template <bool QOUT, bool I8, bool SPLITK, bool RSB>
+template <bool QOUT, bool I8, bool SPLITK, bool RSB, bool F32 = false>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
@@ -460,6 +461,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     }
                 }
             };
+            // the unrounded-output build: fp32(alpha * acc) + bias in fp32, stored as is
+            auto store_f32 = [&](const uint32_t (&r)[32], int n0) {
+                const int row = row0 + lane;
+                if (n0 >= p.N || row >= p.M) return;
+                float* yrow = p.y32 + (size_t)row * p.N;
+                const uint32_t* bw = sbias + (n0 - n_half) / 2;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    float v = __fmul_rn(alpha, __uint_as_float(r[j]));
+                    if (p.bias) v = __fadd_rn(v, (j & 1) ? bf16hi(bw[j / 2]) : bf16lo(bw[j / 2]));
+                    if (n0 + j < p.N) yrow[n0 + j] = v;
+                }
+            };
             // Two chunks at a time: both tensor-memory loads are in flight together, and
             // the columns are released as soon as they are in registers -- the shared
             // columns first, so the next tile's MMAs start before this tile is stored.
@@ -497,6 +511,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     continue;
                 }
                 const int n00 = n_blk * BN + c0 * 32, n01 = n_blk * BN + c1 * 32;
+                if constexpr (F32) {
+                    store_f32(r0, n00);
+                    store_f32(r1, n01);
+                    continue;
+                }
                 uint32_t w0[16], w1[16];
                 if (n00 < p.N) make_words(r0, n00, w0);   // warp-uniform
                 if (n01 < p.N) make_words(r1, n01, w1);
@@ -566,6 +585,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         v[j] = __fadd_rn(v[j], __uint_as_float((uint32_t)p.bias[min(col + j, p.N - 1)] << 16));
+                }
+                if constexpr (F32) {
+                    float* yp32 = p.y32 + (size_t)(m_blk * BM + row) * p.N + col;
+                    for (int j = 0; j < 4 && col + j < p.N; ++j) yp32[j] = v[j];
+                    continue;
                 }
                 const uint32_t lo = bf16x2_bits(v[0], v[1]), hi = bf16x2_bits(v[2], v[3]);
                 uint16_t* yp = p.y + (size_t)(m_blk * BM + row) * p.N + col;
@@ -647,11 +671,11 @@ cudaLaunchConfig_t split_k_config(int grid, int splits, cudaStream_t stream,
     return cfg;
 }
 
-template <bool RSB>
+template <bool RSB, bool F32>
 bool split_k_attr(int device) {
     static std::atomic<int> done[64];
     if (done[device & 63].load(std::memory_order_acquire)) return true;
-    if (cudaFuncSetAttribute(gemm_kernel<false, false, true, RSB>,
+    if (cudaFuncSetAttribute(gemm_kernel<false, false, true, RSB, F32>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmSmem<RSB>::BYTES) != cudaSuccess)
         return false;
@@ -662,10 +686,10 @@ bool split_k_attr(int device) {
 // K splits for a grid with too few tiles to fill the SMs: the largest S <= 8 (a portable
 // cluster) with S <= ceil(K / 256) and tiles * S <= SMs whose clusters are all resident
 // at once (cudaOccupancyMaxActiveClusters, cached per device and S); 1 = no split.
-template <bool RSB>
+template <bool RSB, bool F32>
 int choose_splits(int tiles, int k_tiles, const DeviceInfo& dev) {
     if (tiles * 2 > dev.sms || k_tiles < 2) return 1;
-    if (!split_k_attr<RSB>(dev.device)) return 1;
+    if (!split_k_attr<RSB, F32>(dev.device)) return 1;
     static std::atomic<int> cap[64][9];   // max active clusters + 1 (0 = not queried yet)
     const int smax = min(8, min(k_tiles, dev.sms / tiles));
     for (int sp = smax; sp >= 2; --sp) {
@@ -674,7 +698,7 @@ int choose_splits(int tiles, int k_tiles, const DeviceInfo& dev) {
             cudaLaunchAttribute attr[2];
             const cudaLaunchConfig_t cfg = split_k_config<RSB>(sp * tiles, sp, nullptr, attr);
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<false, false, true, RSB>, &cfg) !=
+            if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<false, false, true, RSB, F32>, &cfg) !=
                 cudaSuccess) {
                 (void)cudaGetLastError();
                 n = 0;
@@ -687,13 +711,13 @@ int choose_splits(int tiles, int k_tiles, const DeviceInfo& dev) {
     return 1;
 }
 
-template <bool RSB>
+template <bool RSB, bool F32>
 nvfp4_status launch_split_k(const CUtensorMap& mapA, const CUtensorMap& mapB,
                             const CUtensorMap& mapY, const GemmParams& p, int grid, int splits,
                             cudaStream_t stream) {
     cudaLaunchAttribute attr[2];
     const cudaLaunchConfig_t cfg = split_k_config<RSB>(grid, splits, stream, attr, true);
-    if (cudaLaunchKernelEx(&cfg, gemm_kernel<false, false, true, RSB>, mapA, mapB, mapY, p) !=
+    if (cudaLaunchKernelEx(&cfg, gemm_kernel<false, false, true, RSB, F32>, mapA, mapB, mapY, p) !=
         cudaSuccess)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
@@ -701,8 +725,9 @@ nvfp4_status launch_split_k(const CUtensorMap& mapA, const CUtensorMap& mapB,
 
 // One launcher for the builds of the kernel: NVFP4 (sfa = 128x4 scales; sfb = 128x4
 // scales, or with RSB the prepared weight scales; alpha), NVFP4 with the quantized
-// output, and int8 (sfa/sfb unused; sx/sw = fp32 row scales of A and B).
-template <bool QOUT, bool I8, bool RSB = false>
+// output, int8 (sfa/sfb unused; sx/sw = fp32 row scales of A and B), and (F32) the
+// NVFP4 GEMM with an unrounded fp32 output y.
+template <bool QOUT, bool I8, bool RSB = false, bool F32 = false>
 nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                               const uint8_t* sfb, const float* alpha, const void* bias, void* y,
                               int64_t M, int64_t N, int64_t K, const QuantOut* q,
@@ -717,20 +742,20 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
     CUtensorMap mapA, mapB, mapY;
     if (!make_operand_map(&mapA, a, M, kbytes, BM) || !make_operand_map(&mapB, b, N, kbytes, BN))
         return NVFP4_ERR_CUDA;
-    const bool tma_store = !QOUT && (N % 8) == 0;
+    const bool tma_store = !QOUT && !F32 && (N % 8) == 0;
     if (tma_store) {
         if (!make_output_map(&mapY, y, M, N)) return NVFP4_ERR_CUDA;
     } else {
         mapY = mapA;   // unused
     }
 
-    static bool attr_set[64] = {false};
-    if (!attr_set[dev.device & 63]) {
-        if (cudaFuncSetAttribute(gemm_kernel<QOUT, I8, false, RSB>,
+    static std::atomic<int> attr_set[64];
+    if (!attr_set[dev.device & 63].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(gemm_kernel<QOUT, I8, false, RSB, F32>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  GemmSmem<RSB>::BYTES) != cudaSuccess)
             return NVFP4_ERR_CUDA;
-        attr_set[dev.device & 63] = true;
+        attr_set[dev.device & 63].store(1, std::memory_order_release);
     }
 
     GemmParams p{};
@@ -738,7 +763,8 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
     p.sfb = sfb;
     p.alpha = alpha;
     p.bias = static_cast<const uint16_t*>(bias);
-    p.y = static_cast<uint16_t*>(y);
+    p.y = F32 ? nullptr : static_cast<uint16_t*>(y);
+    p.y32 = F32 ? static_cast<float*>(y) : nullptr;
     p.M = (int)M;
     p.N = (int)N;
     p.m_blocks = (int)((M + BM - 1) / BM);
@@ -764,10 +790,10 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
 
     const int tiles = p.m_blocks * p.n_blocks;
     if constexpr (!QOUT && !I8) {
-        const int splits = choose_splits<RSB>(tiles, p.k_tiles, dev);
+        const int splits = choose_splits<RSB, F32>(tiles, p.k_tiles, dev);
         if (splits > 1) {
             p.splits = splits;
-            return launch_split_k<RSB>(mapA, mapB, mapY, p, tiles * splits, splits, stream);
+            return launch_split_k<RSB, F32>(mapA, mapB, mapY, p, tiles * splits, splits, stream);
         }
         // One full wave plus a short second one (at most SMs / 2 tiles) of long tiles
         // (K >= 4096): the full wave runs persistent, the leftover tiles split K over
@@ -776,23 +802,23 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
         // it replaces only the last of many waves or a short-K wave.
         const int tail = tiles % dev.sms;
         if (tiles > dev.sms && tiles < 2 * dev.sms && tail > 0 && p.k_tiles >= 16) {
-            const int ts = choose_splits<RSB>(tail, p.k_tiles, dev);
+            const int ts = choose_splits<RSB, F32>(tail, p.k_tiles, dev);
             if (ts > 1) {
                 GemmParams full = p;
                 full.tile_count = tiles - tail;
-                if (launch_pdl(gemm_kernel<false, false, false, RSB>, (unsigned)dev.sms, THREADS,
+                if (launch_pdl(gemm_kernel<false, false, false, RSB, F32>, (unsigned)dev.sms, THREADS,
                                GemmSmem<RSB>::BYTES, stream, mapA, mapB, mapY, full) != cudaSuccess)
                     return NVFP4_ERR_CUDA;
                 GemmParams rest = p;
                 rest.tile_base = tiles - tail;
                 rest.tile_count = tail;
                 rest.splits = ts;
-                return launch_split_k<RSB>(mapA, mapB, mapY, rest, tail * ts, ts, stream);
+                return launch_split_k<RSB, F32>(mapA, mapB, mapY, rest, tail * ts, ts, stream);
             }
         }
     }
     const int grid = tiles < dev.sms ? tiles : dev.sms;
-    if (launch_pdl(gemm_kernel<QOUT, I8, false, RSB>, (unsigned)grid, THREADS,
+    if (launch_pdl(gemm_kernel<QOUT, I8, false, RSB, F32>, (unsigned)grid, THREADS,
                    GemmSmem<RSB>::BYTES, stream, mapA, mapB, mapY, p) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
@@ -855,6 +881,17 @@ nvfp4_status launch_gemm_prepared(const uint8_t* a, const uint8_t* sfa, const ui
                                   cudaStream_t stream) {
     return launch_gemm_impl<false, false, true>(a, sfa, b, sfb_prepared, alpha, bias, y, M, N, K,
                                                 nullptr, nullptr, nullptr, stream);
+}
+
+nvfp4_status launch_gemm_f32(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                             const uint8_t* sfb, bool sfb_prepared, const float* alpha,
+                             const void* bias, float* y, int64_t M, int64_t N, int64_t K,
+                             cudaStream_t stream) {
+    if (sfb_prepared)
+        return launch_gemm_impl<false, false, true, true>(a, sfa, b, sfb, alpha, bias, y, M, N,
+                                                          K, nullptr, nullptr, nullptr, stream);
+    return launch_gemm_impl<false, false, false, true>(a, sfa, b, sfb, alpha, bias, y, M, N, K,
+                                                       nullptr, nullptr, nullptr, stream);
 }
 
 nvfp4_status launch_gemm_quant_out(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,

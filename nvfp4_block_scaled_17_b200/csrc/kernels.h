@@ -64,6 +64,13 @@ size_t prepared_scale_bytes(int64_t N, int64_t K);
 nvfp4_status launch_prepare_scales(const uint8_t* sf, int64_t N, int64_t K, uint8_t* out,
                                    cudaStream_t stream);
 
+// The same GEMM (128x4 or prepared weight scales) with an unrounded fp32 output:
+// y[m, n] = fp32(alpha * acc) + bias[n], the value the bf16 builds round once.
+nvfp4_status launch_gemm_f32(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                             const uint8_t* sfb, bool sfb_prepared, const float* alpha,
+                             const void* bias, float* y, int64_t M, int64_t N, int64_t K,
+                             cudaStream_t stream);
+
 // The GEMM whose epilogue emits the NVFP4 encoding of its bf16 output instead of the
 // output itself (static global scale gsf_out, 128x4 scales, N % 64 == 0).
 nvfp4_status launch_gemm_quant_out(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,

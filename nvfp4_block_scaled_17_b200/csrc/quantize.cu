@@ -16,6 +16,7 @@
 // (one shuffle per value); stages 1, 2, 4 stay inside a chunk and 16, 32, 64 inside
 // a lane.  Block maxima need one shuffle per block; the scale bytes of four blocks
 // form one aligned 32-bit word of the 128x4 layout.
+#include <atomic>
 #include <cmath>
 
 #include "common.cuh"
@@ -726,13 +727,13 @@ nvfp4_status launch_single_pass(const CUtensorMap& map, const UnitParams& p, con
                                 int grid, float* partials, int device, int* status,
                                 cudaStream_t stream) {
     constexpr int smem = TmaShape<G>::SMEM;
-    static bool attr_set[64] = {false};
+    static std::atomic<int> attr_set[64];
     if (device < 0 || device >= 64) return NVFP4_ERR_DEVICE;
-    if (!attr_set[device]) {
+    if (!attr_set[device].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(single_pass_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem) != cudaSuccess)
             return NVFP4_ERR_CUDA;
-        attr_set[device] = true;
+        attr_set[device].store(1, std::memory_order_release);
     }
     // the arrival counter lives in the last word of the caller's 4 KiB workspace
     unsigned int* arrive = reinterpret_cast<unsigned int*>(partials) + (kMaxPartials - 1);
@@ -784,13 +785,13 @@ template <int G, int MODE>
 nvfp4_status launch_tma_unit(const CUtensorMap& map, const UnitParams& p, const TmaParams& t,
                              int grid, int device, int* status, cudaStream_t stream) {
     constexpr int smem = TmaShape<G>::SMEM;
-    static bool attr_set[64] = {false};
+    static std::atomic<int> attr_set[64];
     if (device < 0 || device >= 64) return NVFP4_ERR_DEVICE;
-    if (!attr_set[device]) {
+    if (!attr_set[device].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(tma_unit_kernel<G, MODE>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return NVFP4_ERR_CUDA;
-        attr_set[device] = true;
+        attr_set[device].store(1, std::memory_order_release);
     }
     if (launch_pdl(tma_unit_kernel<G, MODE>, (unsigned)grid, kTmaThreads, smem, stream, map, p, t,
                    status) != cudaSuccess)

@@ -111,6 +111,11 @@ def test_gemm_and_linear_argument_errors(L):
     assert pw(A, -1, 64, A, S) == nv.ERR_INVALID_ARG
     assert pw(A, 256, 96, A, S) == nv.ERR_SHAPE
     assert pw(A, 256, 64, MIS, S) == nv.ERR_ALIGN
+    df = L.nvfp4_debug_gemm_f32
+    assert df(A, A, A, A, 0, A, None, A, 4, 4, 48, S) == nv.ERR_SHAPE         # K % 64
+    assert df(A, A, A, A, 2, A, None, A, 4, 4, 64, S) == nv.ERR_INVALID_ARG   # prepared flag
+    assert df(A, A, A, A, 1, None, None, A, 4, 4, 64, S) == nv.ERR_INVALID_ARG
+    assert df(A, A, A, A, 0, A, None, MIS, 4, 4, 64, S) == nv.ERR_ALIGN
     lp = L.nvfp4_linear_prepared
     assert lp(A, 4, 64, A, A, A, 8, None, None, 0, A, 16, A, S) == nv.ERR_WORKSPACE
     assert lp(A, 4, 96, A, A, A, 8, None, None, 0, A, 1 << 20, A, S) == nv.ERR_SHAPE

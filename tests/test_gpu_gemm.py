@@ -13,7 +13,7 @@ import torch
 
 import nvfp4_block_scaled_17_b200 as nv
 from nvfp4_block_scaled_17_b200 import workloads as W
-from gpu_util import assert_gemm_close, to_np
+from gpu_util import assert_gemm_close, assert_gemm_strict, rounds_to, to_np
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -86,6 +86,43 @@ def test_gemm_split_k(oracle, M, N, K, rows, cols):
     sel = None if rows is None else sample_rows(M, rows, seed=M + N)
     csel = None if cols is None else sample_rows(N, cols, seed=N + K)
     run_gemm_case(oracle, M, N, K, bias=True, seed=M * 13 + N + K, rows=sel, cols=csel)
+
+
+@pytest.mark.parametrize("prepared", [False, True], ids=["128x4", "prepared"])
+@pytest.mark.parametrize("M,N,K", [
+    (128, 256, 256), (1, 8, 64), (100, 200, 192), (129, 300, 320), (257, 513, 1024),
+    (384, 256, 2048),
+    (16, 5120, 5120), (7, 2050, 768), (130, 520, 1536),     # split-K over a cluster
+    (1024, 5120, 5120),                                     # full wave + split last wave
+    (2048, 3072, 1024),                                     # persistent, several waves
+])
+def test_gemm_f32_strict(oracle, M, N, K, prepared):
+    """The unrounded output of the same GEMM (nvfp4_debug_gemm_f32) within both stated
+    bounds without widening, and the bf16 output of nvfp4_gemm / nvfp4_gemm_prepared
+    equal to it rounded to nearest even."""
+    seed = M * 17 + N * 3 + K
+    x = W.with_outliers((M, K), 0.01, 20.0, W._gen(seed, "cpu"), "cpu")
+    w = W.normal((N, K), 0.02, W._gen(seed + 1, "cpu"), "cpu").to(torch.bfloat16)
+    b = W.normal((N,), 0.01, W._gen(seed + 2, "cpu"), "cpu").to(torch.bfloat16)
+    xp, xsf, gx = oracle.quantize(W.to_u16(x))
+    wp, wsf, gw = oracle.quantize(W.to_u16(w))
+    al = oracle.alpha(gx, gw)
+    alpha = torch.tensor([al], device=DEV)
+    wsf_d = t(wsf)
+    if prepared:
+        wsf_d = nv.prepare_weight_scales(wsf_d, N, K)
+        y = nv.nvfp4_gemm_prepared(t(xp), t(xsf), t(wp), wsf_d, alpha, b.to(DEV), M, N, K)
+    else:
+        y = nv.nvfp4_gemm(t(xp), t(xsf), t(wp), wsf_d, alpha, b.to(DEV), M, N, K)
+    y32 = nv.nvfp4_debug_gemm_f32(t(xp), t(xsf), t(wp), wsf_d, alpha, b.to(DEV), M, N, K,
+                                  prepared=prepared)
+    torch.cuda.synchronize()
+    assert nv.last_device_status() == nv.OK
+    assert rounds_to(y32, y)
+    rows = None if M <= 256 else sample_rows(M, 256, seed=M)
+    y64 = oracle.gemm_f64(xp, xsf, wp, wsf, M, N, K, al, W.to_u16(b), rows=rows)
+    yg = y32 if rows is None else y32[torch.from_numpy(rows).to(DEV)]
+    assert_gemm_strict(yg, y64, f"gemm {M}x{N}x{K} {'prepared' if prepared else '128x4'}")
 
 
 def test_gemm_split_k_deterministic_and_graph_capturable():
@@ -170,19 +207,6 @@ def test_linear_parity(oracle, group, dynamic, M, N, K):
     y64, *_ = oracle.linear(W.to_u16(x), owp, owsf, ogw, N, W.to_u16(b), gsf_x=gsf_x,
                             rotate_group=group)
     assert_gemm_close(y, y64, f"linear g={group} dynamic={dynamic}")
-
-
-def test_linear_vit_block_full_size(oracle):
-    """The four ViT-block linears at the 8-tile batch, g = 128, dynamic scale; sampled rows."""
-    for lin in W.vit_block("cpu"):
-        wp, wsf, gw = nv.pack_weight(lin.weight.to(DEV), 128)
-        y = nv.nvfp4_linear(lin.x.to(DEV), wp, wsf, gw, lin.N, bias=lin.bias.to(DEV),
-                            rotate_group=128)
-        torch.cuda.synchronize()
-        rows = sample_rows(lin.x.shape[0], 24, seed=lin.N)
-        y64, *_ = oracle.linear(W.to_u16(lin.x), to_np(wp), to_np(wsf), float(gw.item()), lin.N,
-                                W.to_u16(lin.bias), rotate_group=128, rows=rows)
-        assert_gemm_close(y[torch.from_numpy(rows).to(DEV)], y64, lin.name)
 
 
 def test_probe_error_on_gpu():
