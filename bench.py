@@ -67,8 +67,8 @@ MEASURED_TRAFFIC = {
 
 GROUP = 128
 TOKENS = 8 * 4096
-CPU_SAMPLE_ROWS = 2048
-REF_SAMPLE_ROWS = 256
+CPU_SAMPLE_ROWS = 16384
+REF_SAMPLE_ROWS = 1024
 
 
 def measured_traffic(key):
@@ -314,13 +314,14 @@ def timed_steps(layers, dynamic, steps, warmup, dist_on):
 
 def quantizer_launches(M, K, group, dynamic, sms=148):
     """Kernel launches one nvfp4_quantize call makes: the encode pass, plus the amax pass
-    for a dynamic scale unless the call fits the single-pass kernel (every warp of 16 per
-    SM holding at most 3 items of 16 units)."""
+    for a dynamic scale unless the call fits the single-pass kernel (rows of whole
+    128-value units, 12 warps per SM each holding at most 2 items of 32 units)."""
     if not dynamic:
         return 1
-    unit = 128 if group == 128 else 64
-    items = -(-(M * (K // unit)) // (16 if group == 128 else 32))
-    return 1 if items <= sms * 16 * 3 else 2
+    if K % 128:
+        return 2
+    items = -(-(M * (K // 128)) // 32)
+    return 1 if items <= sms * 12 * 2 else 2
 
 
 def max_over_ranks(v: float, dist_on: bool) -> float:

@@ -610,21 +610,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     }
 }
 
-// 2-D uint8 view [rows, row_bytes] with a [box_rows, 128-byte] box, 128-byte swizzle.
-bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes,
-                      int box_rows) {
-    auto enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-    cuuint32_t box[2] = {(cuuint32_t)BKB, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 // bf16 [M, N] output with a 32 x 32 box and 64-byte swizzle (N % 8 == 0).
 bool make_output_map(CUtensorMap* map, void* base, int64_t M, int64_t N) {
     auto enc = tensor_map_encoder();
@@ -640,6 +625,21 @@ bool make_output_map(CUtensorMap* map, void* base, int64_t M, int64_t N) {
 }
 
 }  // namespace
+
+// 2-D uint8 view [rows, row_bytes] with a [box_rows, 128-byte] box, 128-byte swizzle.
+bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes,
+                      int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)BKB, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 namespace {
 
@@ -738,6 +738,11 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
     int* status = nullptr;
     if ((st = status_word(&status)) != NVFP4_OK) return st;
 
+    // few activation rows: the swapped-operand kernel (gemm_small.cu)
+    if constexpr (!QOUT && !I8) {
+        if (M <= kSmallMaxRows)
+            return launch_gemm_small(a, sfa, b, sfb, RSB, F32, alpha, bias, y, M, N, K, stream);
+    }
     const int64_t kbytes = I8 ? K : K / 2;   // bytes of one operand row
     CUtensorMap mapA, mapB, mapY;
     if (!make_operand_map(&mapA, a, M, kbytes, BM) || !make_operand_map(&mapB, b, N, kbytes, BN))
@@ -790,6 +795,7 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
 
     const int tiles = p.m_blocks * p.n_blocks;
     if constexpr (!QOUT && !I8) {
+
         const int splits = choose_splits<RSB, F32>(tiles, p.k_tiles, dev);
         if (splits > 1) {
             p.splits = splits;

@@ -1,0 +1,409 @@
+// gemm_small.cu -- the block-scaled FP4 GEMM for few activation rows (M <= 128).
+//
+// Pages: "minimax_h3_nvfp4_decoder" -- nvfp4_linear_inference (mm_fp4 with alpha =
+// 1/(global_sf_x * global_sf_w), bf16 output, then the bias); the operation is the one
+// gemm.cu computes: y[m, n] = bf16(fp32(alpha * acc) + bias[n]).
+//
+// With M of 16 or 128 rows (a decode step, or the Qwen3-VL projections at small batch)
+// the output has too few 128-row tiles to fill the tensor cores: an M = 128 MMA would
+// spend 7/8 of its work on padding rows, and the weight stream (N x K / 2 bytes, read
+// once) is what bounds the call.  So the operands swap: the tensor cores compute
+// y^T = W x^T, 128 weight rows filling the MMA's M and the activation rows the MMA's N
+// (M rounded up to a multiple of 16).
+//
+// Design (320 threads, one CTA per SM):
+//   * a tile is 256 weight rows (output columns), two M = 128 MMAs per K step sharing
+//     the activation operand; K is split over the S CTAs of a thread-block cluster,
+//     S chosen so that every tile's cluster is resident at once;
+//   * warp 0 loads, per 256-value K stage, the 256 x 128-byte weight box and the
+//     M x 128-byte activation box (128-byte swizzle, rows past M zero-filled), the
+//     activation's 128x4 scale chunks and the weight's: the 128x4 chunks of both row
+//     tiles, or, from prepared weight scales, the first 1 KiB of each step's 4 KiB
+//     slot, which holds both tiles' 128-byte pieces 256 bytes apart (the copy below
+//     reads them with a 256-byte stride, so no replicated bytes cross HBM);
+//   * warp 1 copies each K step's three scale chunks into a five-slot tensor-memory
+//     ring and issues the two MMAs (kind::mxf4nvf4, block16, M = 128, N = M padded);
+//   * warps 2..9 move the two fp32 partial accumulators into shared memory (the idle
+//     stage buffers), then, after a cluster barrier, each CTA sums its share of the
+//     tile over the S partials in rank order (distributed shared memory) and applies
+//     alpha and the bias: deterministic, and the unrounded-output build (F32) stores
+//     the same fp32 value the bf16 build rounds.
+// Every wait is bounded; on expiry the kernel records NVFP4_ERR_TIMEOUT, drains its
+// copies and MMAs, frees tensor memory and returns.  No load uses cluster multicast.
+#include <atomic>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr int XW_ROWS = 256;                 // weight rows per tile (two MMAs)
+constexpr int XBKB = 128;                    // packed K bytes per stage (256 values)
+constexpr int XSTAGES = 4;
+constexpr int XMAX = 128;                    // activation rows at most (the MMA's N)
+constexpr int XTHREADS = 320;
+constexpr int XS_W = XW_ROWS * XBKB;         // 32 KiB
+constexpr int XS_X = XMAX * XBKB;            // 16 KiB
+constexpr int XS_SFW = 4096;                 // two row tiles x four steps x 512 B (or 4 x 1 KiB)
+constexpr int XS_SFX = 2048;                 // four steps x 512 B
+constexpr int XS_STAGE = XS_W + XS_X + XS_SFW + XS_SFX;
+constexpr int XSMEM = 1024 + XSTAGES * XS_STAGE + 256;
+static_assert(XSMEM <= 232448, "dynamic shared memory above the 227 KiB a CTA can have");
+static_assert(XMAX * XW_ROWS * 4 <= XSTAGES * XS_STAGE, "partial tile must fit the stages");
+constexpr int XTMEM_COLS = 512;
+constexpr uint32_t XTMEM_ACC1 = 128;         // second accumulator (weight rows 128..255)
+constexpr uint32_t XTMEM_SF = 256;           // scale ring: 5 slots x 12 columns
+constexpr int XSF_SLOTS = 5;
+
+struct SmallParams {
+    const uint8_t* sfw;        // weight scales: 128x4, or prepared (RSB)
+    const uint8_t* sfx;        // activation 128x4 scales
+    const float* alpha;
+    const uint16_t* bias;      // bf16 [N] or null
+    uint16_t* y;               // bf16 [M, N]
+    float* y32;                // fp32 [M, N] (the unrounded-output build)
+    int M, N;
+    int mpad;                  // the MMA's N: M rounded up to 16
+    uint32_t idesc;
+    int k_tiles;               // ceil(K / 256)
+    int kchunks;               // K / 64
+    int w_row_tiles;           // ceil(N / 128)
+    int splits;
+    int* status;
+    uint64_t budget_ns;
+};
+
+// tcgen05.cp source of a 32-row x 16-byte block whose 8-row core matrices are `stride`
+// bytes apart (128 for a contiguous 128x4 chunk, 256 for a piece of a prepared slot).
+__device__ __forceinline__ uint64_t sdesc_sf_stride(uint32_t smem_addr, uint32_t stride) {
+    return (uint64_t)((smem_addr >> 4) & 0x3fffu) | ((uint64_t)(stride >> 4) << 32) |
+           ((uint64_t)1 << 46);
+}
+
+template <bool RSB, bool F32>
+__global__ void __launch_bounds__(XTHREADS, 1)
+gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                  const SmallParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + XSTAGES * XS_STAGE);
+    uint64_t* empty = full + XSTAGES;
+    uint64_t* acc_full = empty + XSTAGES;
+    uint64_t* drain = acc_full + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < XSTAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, XTMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    griddep_wait();
+    griddep_launch_dependents();
+
+    const int splits = p.splits;
+    const int rank = (int)cluster_rank();
+    const int tile = (int)blockIdx.x / splits;
+    const int kt_begin = rank * p.k_tiles / splits;
+    const int kt_end = (rank + 1) * p.k_tiles / splits;
+    const bool two = 2 * tile + 1 < p.w_row_tiles;   // the second 128-row MMA has rows
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tensormap(&tmW);
+            prefetch_tensormap(&tmX);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_phase = 0;
+            for (int kt = kt_begin; kt < kt_end; ++kt) {
+                if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, p.budget_ns))
+                    break;
+                uint8_t* sW = smem + stage * XS_STAGE;
+                uint8_t* sX = sW + XS_W;
+                uint8_t* sSFW = sX + XS_X;
+                uint8_t* sSFX = sSFW + XS_SFW;
+                const int steps = min(4, p.kchunks - 4 * kt);
+                const uint32_t sfx_bytes = (uint32_t)steps * 512u;
+                const uint32_t sfw_bytes = RSB ? (uint32_t)steps * 1024u : sfx_bytes * (two ? 2u : 1u);
+                mbar_arrive_expect_tx(&full[stage], XS_W + (uint32_t)p.mpad * XBKB + sfw_bytes + sfx_bytes);
+                tma_load_2d(sW, &tmW, &full[stage], kt * XBKB, tile * XW_ROWS);
+                tma_load_2d(sX, &tmX, &full[stage], kt * XBKB, 0);
+                if constexpr (RSB) {
+                    for (int j = 0; j < steps; ++j)
+                        bulk_load(sSFW + j * 1024,
+                                  p.sfw + ((size_t)tile * p.kchunks + 4 * kt + j) * 4096, 1024u,
+                                  &full[stage]);
+                } else {
+                    for (int t = 0; t < (two ? 2 : 1); ++t)
+                        bulk_load(sSFW + t * 2048,
+                                  p.sfw + ((size_t)(2 * tile + t) * p.kchunks + 4 * kt) * 512,
+                                  sfx_bytes, &full[stage]);
+                }
+                bulk_load(sSFX, p.sfx + (size_t)(4 * kt) * 512, sfx_bytes, &full[stage]);
+                issued |= 1u << stage;
+                issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                if (++stage == XSTAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            // every fill this thread started must land before the block can exit
+            for (int s = 0; s < XSTAGES; ++s)
+                if (issued & (1u << s)) {
+                    volatile int no_abort = 0;
+                    mbar_wait_bounded(&full[s], (issued_phase >> s) & 1, &no_abort, p.status,
+                                      p.budget_ns);
+                }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int slot = 0;
+            bool ok = true;
+            for (int kt = kt_begin; kt < kt_end; ++kt) {
+                if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, p.budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int steps = min(4, p.kchunks - 4 * kt);
+                const uint32_t w0 = smem_u32(smem + stage * XS_STAGE);
+                const uint32_t x0 = w0 + XS_W;
+                const uint32_t sfw0 = x0 + XS_X;
+                const uint32_t sfx0 = sfw0 + XS_SFW;
+                for (int kk = 0; kk < steps; ++kk) {
+                    const uint32_t sf_t = tmem + XTMEM_SF + 12u * (uint32_t)slot;
+                    if constexpr (RSB) {
+                        tc_copy_sf(sf_t, sdesc_sf_stride(sfw0 + 1024 * kk, 256));
+                        if (two) tc_copy_sf(sf_t + 4, sdesc_sf_stride(sfw0 + 1024 * kk + 128, 256));
+                    } else {
+                        tc_copy_sf(sf_t, sdesc_sf_stride(sfw0 + 512 * kk, 128));
+                        if (two) tc_copy_sf(sf_t + 4, sdesc_sf_stride(sfw0 + 2048 + 512 * kk, 128));
+                    }
+                    tc_copy_sf(sf_t + 8, sdesc_sf_stride(sfx0 + 512 * kk, 128));
+                    const uint64_t xdesc = sdesc_kmajor_sw128(x0 + 32 * kk);
+                    const uint32_t acc = (kt > kt_begin || kk > 0) ? 1u : 0u;
+                    mma_nvf4(tmem, sdesc_kmajor_sw128(w0 + 32 * kk), xdesc, p.idesc, sf_t,
+                             sf_t + 8, acc);
+                    if (two)
+                        mma_nvf4(tmem + XTMEM_ACC1, sdesc_kmajor_sw128(w0 + 16384 + 32 * kk), xdesc,
+                                 p.idesc, sf_t + 4, sf_t + 8, acc);
+                    if (++slot == XSF_SLOTS) slot = 0;
+                }
+                tc_commit(&empty[stage]);
+                if (++stage == XSTAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            if (ok) tc_commit(acc_full);
+            tc_commit(drain);
+            volatile int no_abort = 0;
+            mbar_wait_bounded(drain, 0, &no_abort, p.status, p.budget_ns);
+        }
+        __syncwarp();
+    } else {
+        // the fp32 partial of this CTA's K range into shared memory, [m][256] floats:
+        // warp (t, q) holds weight rows t * 128 + 32 q + lane of the tile
+        const int t = (warp - 2) >> 2;
+        const int quad = warp & 3;
+        if ((t == 0 || two) &&
+            mbar_wait_bounded(acc_full, 0, abort_flag, p.status, p.budget_ns)) {
+            tc_fence_after();
+            float* part = reinterpret_cast<float*>(smem);
+            const int nl = t * 128 + quad * 32 + lane;
+            const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + (t ? XTMEM_ACC1 : 0u);
+            for (int c = 0; c * 32 < p.M; ++c) {
+                uint32_t r[32];
+                tmem_ld32(base + (uint32_t)c * 32, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int m = c * 32 + j;
+                    if (m < p.M) part[m * XW_ROWS + nl] = __uint_as_float(r[j]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    // Every thread of the cluster gets here after bounded work, so the barriers below
+    // cannot hang.  Rank r then reduces granules [r G / S, (r + 1) G / S) of the M x 256
+    // partials (4 floats each) in rank order and stores them; the second barrier keeps
+    // every partial alive until all ranks have read it.
+    cluster_sync_all();
+    if (warp >= 2 && !*abort_flag) {
+        const int G = p.M * (XW_ROWS / 4);
+        const int lo = rank * G / splits, hi = (rank + 1) * G / splits;
+        const uint32_t part = smem_u32(smem);
+        const float alpha = *p.alpha;
+        for (int idx = lo + (int)threadIdx.x - 64; idx < hi; idx += XTHREADS - 64) {
+            const int m = idx >> 6, g = idx & 63;
+            const int n = tile * XW_ROWS + 4 * g;
+            if (n >= p.N) continue;
+            const uint32_t off = part + (uint32_t)((m * XW_ROWS + 4 * g) * 4);
+            float4 acc = ld_dsmem_f4(dsmem_addr(off, 0));
+            for (int r = 1; r < splits; ++r) {
+                const float4 v = ld_dsmem_f4(dsmem_addr(off, (uint32_t)r));
+                acc.x = __fadd_rn(acc.x, v.x);
+                acc.y = __fadd_rn(acc.y, v.y);
+                acc.z = __fadd_rn(acc.z, v.z);
+                acc.w = __fadd_rn(acc.w, v.w);
+            }
+            float v[4] = {__fmul_rn(alpha, acc.x), __fmul_rn(alpha, acc.y),
+                          __fmul_rn(alpha, acc.z), __fmul_rn(alpha, acc.w)};
+            if (p.bias) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    v[j] = __fadd_rn(v[j], __uint_as_float((uint32_t)p.bias[min(n + j, p.N - 1)] << 16));
+            }
+            if constexpr (F32) {
+                float* yp = p.y32 + (size_t)m * p.N + n;
+                for (int j = 0; j < 4 && n + j < p.N; ++j) yp[j] = v[j];
+            } else {
+                const uint32_t lo2 = bf16x2_rn(v[0], v[1]), hi2 = bf16x2_rn(v[2], v[3]);
+                uint16_t* yp = p.y + (size_t)m * p.N + n;
+                if ((p.N & 3) == 0) {
+                    *reinterpret_cast<uint2*>(yp) = make_uint2(lo2, hi2);
+                } else {
+                    const uint16_t hv[4] = {(uint16_t)lo2, (uint16_t)(lo2 >> 16), (uint16_t)hi2,
+                                            (uint16_t)(hi2 >> 16)};
+                    for (int j = 0; j < 4 && n + j < p.N; ++j) yp[j] = hv[j];
+                }
+            }
+        }
+    }
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, XTMEM_COLS);
+    }
+}
+
+cudaLaunchConfig_t small_config(int grid, int splits, cudaStream_t stream,
+                                cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(XTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = XSMEM;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cfg;
+}
+
+template <bool RSB, bool F32>
+bool small_attr(int device) {
+    static std::atomic<int> done[64];
+    if (done[device & 63].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(gemm_small_kernel<RSB, F32>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, XSMEM) != cudaSuccess)
+        return false;
+    done[device & 63].store(1, std::memory_order_release);
+    return true;
+}
+
+// K splits: the largest S <= 8 (a portable cluster) with S <= the K stages and
+// tiles * S <= SMs whose clusters are all resident at once (cached per device and S).
+template <bool RSB, bool F32>
+int small_splits(int tiles, int k_tiles, const DeviceInfo& dev) {
+    static std::atomic<int> cap[64][9];   // max active clusters + 1 (0 = not queried yet)
+    int smax = min(8, k_tiles);
+    if (tiles * smax > dev.sms) smax = max(1, dev.sms / tiles);
+    for (int sp = smax; sp >= 2; --sp) {
+        int c = cap[dev.device & 63][sp].load(std::memory_order_relaxed) - 1;
+        if (c < 0) {
+            cudaLaunchAttribute attr[2];
+            const cudaLaunchConfig_t cfg = small_config(sp * tiles, sp, nullptr, attr);
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, gemm_small_kernel<RSB, F32>, &cfg) != cudaSuccess) {
+                (void)cudaGetLastError();
+                n = 0;
+            }
+            c = n;
+            cap[dev.device & 63][sp].store(c + 1, std::memory_order_relaxed);
+        }
+        if (c >= tiles) return sp;
+    }
+    return 1;
+}
+
+template <bool RSB, bool F32>
+nvfp4_status launch_small_impl(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                               const uint8_t* sfb, const float* alpha, const void* bias, void* y,
+                               int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    DeviceInfo dev;
+    nvfp4_status st = device_info(&dev);
+    if (st != NVFP4_OK) return st;
+    int* status = nullptr;
+    if ((st = status_word(&status)) != NVFP4_OK) return st;
+    if (!small_attr<RSB, F32>(dev.device)) return NVFP4_ERR_CUDA;
+
+    SmallParams p{};
+    p.mpad = (int)((M + 15) / 16 * 16);
+    CUtensorMap mapW, mapX;
+    if (!make_operand_map(&mapW, b, N, K / 2, XW_ROWS) || !make_operand_map(&mapX, a, M, K / 2, p.mpad))
+        return NVFP4_ERR_CUDA;
+    p.sfw = sfb;
+    p.sfx = sfa;
+    p.alpha = alpha;
+    p.bias = static_cast<const uint16_t*>(bias);
+    p.y = F32 ? nullptr : static_cast<uint16_t*>(y);
+    p.y32 = F32 ? static_cast<float*>(y) : nullptr;
+    p.M = (int)M;
+    p.N = (int)N;
+    // E2M1 x E2M1, UE4M3 block scales, both K-major; N = padded M, M = 128
+    p.idesc = (1u << 7) | (1u << 10) | ((uint32_t)(p.mpad >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+    p.k_tiles = (int)((K / 2 + XBKB - 1) / XBKB);
+    p.kchunks = (int)(K / 64);
+    p.w_row_tiles = (int)((N + 127) / 128);
+    p.status = status;
+    p.budget_ns = 4000000000ull;   // 4 s
+    const int tiles = (int)((N + XW_ROWS - 1) / XW_ROWS);
+    p.splits = small_splits<RSB, F32>(tiles, p.k_tiles, dev);
+    cudaLaunchAttribute attr[2];
+    const cudaLaunchConfig_t cfg = small_config(tiles * p.splits, p.splits, stream, attr);
+    if (cudaLaunchKernelEx(&cfg, gemm_small_kernel<RSB, F32>, mapW, mapX, p) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+nvfp4_status launch_gemm_small(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                               const uint8_t* sfb, bool sfb_prepared, bool f32_out,
+                               const float* alpha, const void* bias, void* y, int64_t M,
+                               int64_t N, int64_t K, cudaStream_t stream) {
+    if (M < 1 || M > XMAX) return NVFP4_ERR_INVALID_ARG;
+    if (sfb_prepared)
+        return f32_out ? launch_small_impl<true, true>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream)
+                       : launch_small_impl<true, false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream);
+    return f32_out ? launch_small_impl<false, true>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream)
+                   : launch_small_impl<false, false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream);
+}
+
+}  // namespace nvfp4

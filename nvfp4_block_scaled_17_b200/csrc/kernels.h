@@ -71,6 +71,21 @@ nvfp4_status launch_gemm_f32(const uint8_t* a, const uint8_t* sfa, const uint8_t
                              const void* bias, float* y, int64_t M, int64_t N, int64_t K,
                              cudaStream_t stream);
 
+// The GEMM for M <= kSmallMaxRows activation rows with the operands swapped
+// (y^T = W x^T: weight rows on the MMA's M, activation rows on its N), K split over a
+// thread-block cluster; same arguments and result as launch_gemm / launch_gemm_prepared
+// (sfb_prepared) / launch_gemm_f32 (f32_out, y is then float*).
+constexpr int64_t kSmallMaxRows = 128;
+nvfp4_status launch_gemm_small(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
+                               const uint8_t* sfb, bool sfb_prepared, bool f32_out,
+                               const float* alpha, const void* bias, void* y, int64_t M,
+                               int64_t N, int64_t K, cudaStream_t stream);
+
+// 2-D uint8 tensor map [rows, row_bytes] with a [box_rows, 128-byte] box and the
+// 128-byte swizzle (the GEMM operand loads).
+bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes,
+                      int box_rows);
+
 // The GEMM whose epilogue emits the NVFP4 encoding of its bf16 output instead of the
 // output itself (static global scale gsf_out, 128x4 scales, N % 64 == 0).
 nvfp4_status launch_gemm_quant_out(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,

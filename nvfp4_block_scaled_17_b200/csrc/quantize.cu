@@ -8,14 +8,19 @@
 // "convert_minimax_h3_text_encoder_nvfp4.py" -- quantize_language_linear (weights go
 // through the same quantizer with their own global scale).
 //
-// Work decomposition.  A "unit" is E consecutive values of one row (E = 64, or 128
-// for a 128-wide rotation), handled by a pair of adjacent lanes: lane h of the pair
-// owns the 8-value chunks 2i+h of the unit, so every load instruction of a warp
-// reads 16 whole 32-byte sectors and each 16-value block lies half in each lane.
-// With that split the only cross-lane step of the butterfly is the h = 8 stage
-// (one shuffle per value); stages 1, 2, 4 stay inside a chunk and 16, 32, 64 inside
-// a lane.  Block maxima need one shuffle per block; the scale bytes of four blocks
-// form one aligned 32-bit word of the 128x4 layout.
+// Two work decompositions.
+//   * Rows made of whole 128-value units (K % 128 == 0, every workload here): one
+//     thread owns a unit, loaded through the tensor-memory accelerator, and keeps the
+//     whole butterfly, the block maxima and the encoding in its registers (row_kernel,
+//     row_single_kernel below).
+//   * Any other K % 16 == 0 (unit_kernel): a unit is E consecutive values of one row (E
+//     = 64, or 128 for a 128-wide rotation), handled by a pair of adjacent lanes: lane h
+//     of the pair owns the 8-value chunks 2i+h of the unit, so every load instruction of
+//     a warp reads 16 whole 32-byte sectors and each 16-value block lies half in each
+//     lane.  With that split the only cross-lane step of the butterfly is the h = 8 stage
+//     (one shuffle per value); stages 1, 2, 4 stay inside a chunk and 16, 32, 64 inside a
+//     lane.  Block maxima need one shuffle per block; the scale bytes of four blocks form
+//     one aligned 32-bit word of the 128x4 layout.
 #include <atomic>
 #include <cmath>
 
@@ -324,7 +329,8 @@ __device__ __forceinline__ void encode_unit(const uint4 (&w)[UnitShape<G>::NCT],
     }
 }
 
-// MODE 0: amax partials.  MODE 1: quantize.  MODE 2: rotate only (G > 0).
+// Plain-load form for any K % 16 == 0 (the calls whose rows are not whole 128-value
+// units).  MODE 0: amax partials.  MODE 1: quantize.  MODE 2: rotate only (G > 0).
 template <int G, int MODE>
 __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
     constexpr int E = UnitShape<G>::E;
@@ -397,72 +403,228 @@ __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// TMA-fed form (K % 64 == 0): the same per-unit arithmetic, with x staged in
-// shared memory by the tensor-memory accelerator.
+// Row-unit form (K % 128 == 0): one thread owns a unit of 128 consecutive values of a
+// row, so the whole 128-wide butterfly, the block maxima and the encoding stay in its
+// registers: no shuffles and no lane-pair exchanges.
 //
-// x is viewed as a flat 2-D array of 64-value rows (128 bytes each); an item is
-// the 16 units one warp handles (16 or 32 flat rows), loaded as one box with the
-// 128-byte swizzle, so the lane-pair reads below hit 8 distinct 16-byte bank
-// groups per quarter-warp.  Every warp keeps its own ring of kSlots items and
-// issues the load of item k + kSlots as soon as it has read item k into
-// registers, so HBM latency overlaps the arithmetic of the items in between.
-// One CTA of 16 warps per SM, persistent over the items.
+// x is read as units (256 bytes each) through two tensor maps over the same memory with
+// a 256-byte row stride: one for the first 64 values of every unit, one (based 128 bytes
+// further) for the second 64.  An item is 32 consecutive units, one per lane: one 4 KiB
+// box from each map, 128-byte swizzle, so lane t reads row t of each box and the eight
+// lanes of a quarter-warp hit eight distinct 16-byte bank groups.  Every warp keeps its
+// own ring of kRSlots items and issues the load of item k + kRSlots as soon as its lanes
+// have read item k into registers.  One CTA of kRWarps warps per SM, persistent.
 // ---------------------------------------------------------------------------
 
-constexpr int kTmaWarps = 16;
-constexpr int kTmaThreads = kTmaWarps * 32;
-constexpr int kSlots = 3;
-constexpr int kItemRows = 32;                       // flat 64-value rows per item (4 KiB)
+constexpr int kRWarps = 12;
+constexpr int kRThreads = kRWarps * 32;
+constexpr int kRSlots = 2;
+constexpr int kRHalfBytes = 32 * 128;              // one 64-value half of 32 units
+constexpr int kRItemBytes = 2 * kRHalfBytes;       // 8 KiB: 32 units
+constexpr int kRRingBytes = kRWarps * kRSlots * kRItemBytes;
+constexpr int kRSmem = 1024 + kRRingBytes + kRWarps * kRSlots * 8;
 constexpr uint64_t kTmaWaitBudgetNs = 2000000000ull;
+static_assert(kRSmem <= 232448, "dynamic shared memory above the 227 KiB a CTA can have");
 
-template <int G>
-struct TmaShape {
-    static constexpr int E = UnitShape<G>::E;
-    static constexpr int SUBS = 128 / E;                // units per lane pair per item
-    static constexpr int UPI = 16 * SUBS;               // units per item
-    static constexpr int ITEM_BYTES = kItemRows * 128;
-    static constexpr int RING_BYTES = kTmaWarps * kSlots * ITEM_BYTES;
-    static constexpr int SMEM = 1024 + RING_BYTES + kTmaWarps * kSlots * 8;
-};
-
-struct TmaParams {
-    uint32_t total_units;   // rows * K / E  (< 2^31)
-    uint32_t n_items;
-    uint32_t upr;           // units per row
+struct RowParams {
+    uint32_t total_units;   // rows * K / 128  (< 2^31)
+    uint32_t n_items;       // ceil(total_units / 32)
+    uint32_t upr;           // units per row, K / 128
     FastDiv upr_div;
 };
 
-// Unit of the item read by lane pair `pair` in sub-step `sub`.  With 128-value units a
-// pair reads two flat rows; with 64-value units the order 0,2,4,6 | 1,3,5,7 | 8,10,..
-// keeps the four pairs of a quarter-warp on distinct swizzle phases.
-template <int E>
-__device__ __forceinline__ int item_unit(int pair, int sub) {
-    if constexpr (E == 128) return pair;
-    return sub * 16 + ((pair & 8) | ((pair & 3) << 1) | ((pair >> 2) & 1));
+// fp32 bit pattern of bf16(a) (round to nearest even): a goes to the upper half of the
+// packed pair, +0 to the lower half.
+__device__ __forceinline__ float bf16_round(float a) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(a), "f"(0.0f));
+    return __uint_as_float(d);
 }
 
+// Two fp32 values that are bf16-exact back into one bf16 pair (lo in bits 0..15).
+__device__ __forceinline__ uint32_t pack_bf16_pair(float lo, float hi) {
+    return __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x7632);
+}
+
+// Byte address of chunk c (8 values) of lane `lane`'s unit in an item slot.
+__device__ __forceinline__ uint32_t unit_chunk_off(int lane, int c) {
+    return (uint32_t)((c >> 3) * kRHalfBytes + lane * 128 + (((c & 7) ^ (lane & 7)) << 4));
+}
+
+__device__ __forceinline__ void load_unit(const uint8_t* slot, int lane, uint4 (&w)[16]) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) w[c] = *reinterpret_cast<const uint4*>(slot + unit_chunk_off(lane, c));
+}
+
+// The butterfly stages h = 1, 2, 4, ... < STOP of every G-group of the unit in fp32.  The
+// values are held as pairs (2i, 2i + 1): stage 1 works inside each bf16 pair, straight
+// from the words; stage h >= 2 on pairs h / 2 apart (the pair index bit h / 2 clear keeps
+// both partners in one aligned group of 2h <= G values).
+template <int STOP>
+__device__ __forceinline__ void unit_butterfly(const uint4 (&w)[16], float2 (&v)[64]) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        v[4 * c] = pair_sum_diff(w[c].x);
+        v[4 * c + 1] = pair_sum_diff(w[c].y);
+        v[4 * c + 2] = pair_sum_diff(w[c].z);
+        v[4 * c + 3] = pair_sum_diff(w[c].w);
+    }
+#pragma unroll
+    for (int h = 2; h < STOP; h *= 2)
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+            if ((i & (h / 2)) == 0) bfly2(v[i], v[i + h / 2]);
+}
+
+// The unit's values as fp32: rotated (every G-group times H / sqrt(G), rounded to bf16)
+// or, for G = 0, the bf16 input itself.
+template <int G>
+__device__ __forceinline__ void unit_values(const uint4 (&w)[16], float hscale, float (&r)[128]) {
+    if constexpr (G == 0) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const uint32_t q[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                r[8 * c + 2 * k] = bf16lo(q[k]);
+                r[8 * c + 2 * k + 1] = bf16hi(q[k]);
+            }
+        }
+    } else {
+        float2 v[64];
+        unit_butterfly<G>(w, v);
+        const float2 hs = make_float2(hscale, hscale);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            const float2 g = mul2(v[i], hs);
+            r[2 * i] = bf16_round(g.x);
+            r[2 * i + 1] = bf16_round(g.y);
+        }
+    }
+}
+
+// Running maximum for the amax pass.  G = 0: the bf16 maxima of the words (packed).
+// G > 0: the butterfly up to its last stage, then max(|a| + |b|) over the last stage's
+// pairs -- one of rn(a + b), rn(a - b) has magnitude rn(|a| + |b|) and rounding is
+// monotone, so this is the largest pre-scale magnitude of the rotated values; the
+// rotated bf16 amax is bf16(rn(m * hscale)) of it (rotated_amax_bf16).
+template <int G>
+__device__ __forceinline__ void unit_amax(const uint4 (&w)[16], uint32_t& tmax, float& fmax_) {
+    if constexpr (G == 0) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) tmax = absmax2_bf16(tmax, absmax_word4(w[c]));
+    } else {
+        float2 v[64];
+        unit_butterfly<G / 2>(w, v);
+        constexpr int S = G / 4;   // pair distance of the last stage
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+            if ((i & S) == 0)
+                fmax_ = max3(fmax_, __fadd_rn(fabsf(v[i].x), fabsf(v[i + S].x)),
+                             __fadd_rn(fabsf(v[i].y), fabsf(v[i + S].y)));
+    }
+}
+
+// E4M3 block-scale bytes of two blocks from their scaled maxima y0, y1 >= 0 (or NaN):
+// e4m3_scale_of_scaled_max on each, converted in one instruction; y0's byte is the low one.
+__device__ __forceinline__ uint32_t e4m3_scales2(float y0, float y1) {
+    const float r = __uint_as_float(0x3e2aaaabu);   // rn(1/6)
+    y0 = (y0 > 6000.0f) ? 6000.0f : y0;
+    y1 = (y1 > 6000.0f) ? 6000.0f : y1;
+    const float q0 = __fmul_rn(y0, r), q1 = __fmul_rn(y1, r);
+    const float a0 = __fmaf_rn(__fmaf_rn(-q0, 6.0f, y0), r, q0);
+    const float a1 = __fmaf_rn(__fmaf_rn(-q1, 6.0f, y1), r, q1);
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(a1), "f"(a0));
+    return d;
+}
+
+// max |r[k]| over one 16-value block
+__device__ __forceinline__ float block_absmax16(const float* r) {
+    float m = max3(fabsf(r[0]), fabsf(r[1]), fabsf(r[2]));
+#pragma unroll
+    for (int k = 3; k < 15; k += 2) m = max3(m, fabsf(r[k]), fabsf(r[k + 1]));
+    return fmaxf(m, fabsf(r[15]));
+}
+
+// Encode one unit (values r, bf16-exact): per 16-value block bmax, the E4M3 scale of
+// rn(gsf * bmax) / 6, codes E2M1(rn(x * rn(gsf / scale))), all codes 0 under a zero
+// scale; 64 bytes of packed codes and two scale words of the 128x4 layout.
+__device__ __forceinline__ void encode_unit128(const float (&r)[128], float gsf,
+                                               const float* inv_tab, const UnitParams& p,
+                                               int64_t row, int64_t e0) {
+    uint32_t s8[8];
+#pragma unroll
+    for (int b = 0; b < 8; b += 2) {
+        const uint32_t s = e4m3_scales2(__fmul_rn(gsf, block_absmax16(r + 16 * b)),
+                                        __fmul_rn(gsf, block_absmax16(r + 16 * b + 16)));
+        s8[b] = s & 0xffu;
+        s8[b + 1] = s >> 8;
+    }
+    uint32_t codes[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        const float inv = inv_tab[s8[c >> 1]];   // rn(gsf / dec(s8)); 0 for a zero scale
+        const float2 iv = make_float2(inv, inv);
+        const float* x = r + 8 * c;
+        const float2 a = mul2(make_float2(x[0], x[1]), iv), b = mul2(make_float2(x[2], x[3]), iv);
+        const float2 cc = mul2(make_float2(x[4], x[5]), iv), d = mul2(make_float2(x[6], x[7]), iv);
+        const float q[8] = {a.x, a.y, b.x, b.y, cc.x, cc.y, d.x, d.y};
+        codes[c] = s8[c >> 1] ? e2m1x8_from_f32(q) : 0u;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(p.packed + row * (p.K / 2) + e0 / 2);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        dst[k] = make_uint4(codes[4 * k], codes[4 * k + 1], codes[4 * k + 2], codes[4 * k + 3]);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int64_t cg = e0 / 64 + q;
+        const int64_t off = (((row >> 7) * p.cgroups + cg) << 9) + ((row & 31) << 4) +
+                            (((row >> 5) & 3) << 2);
+        *reinterpret_cast<uint32_t*>(p.sf + off) = s8[4 * q] | (s8[4 * q + 1] << 8) |
+                                                   (s8[4 * q + 2] << 16) | (s8[4 * q + 3] << 24);
+    }
+}
+
+// Scale bytes of the padding rows (rows .. up to the next multiple of 128) are zero.
+template <int THREADS>
+__device__ __forceinline__ void zero_padding_scales(const UnitParams& p) {
+    const int64_t pad_rows = (p.rows + 127) / 128 * 128 - p.rows;
+    for (int64_t i = (int64_t)blockIdx.x * THREADS + threadIdx.x; i < pad_rows * p.cgroups;
+         i += (int64_t)gridDim.x * THREADS) {
+        const int64_t row = p.rows + i / p.cgroups, cg = i % p.cgroups;
+        const int64_t off = (((row >> 7) * p.cgroups + cg) << 9) + ((row & 31) << 4) +
+                            (((row >> 5) & 3) << 2);
+        *reinterpret_cast<uint32_t*>(p.sf + off) = 0u;
+    }
+}
+
+__device__ __forceinline__ void load_item(uint8_t* slot, const CUtensorMap* tmE,
+                                          const CUtensorMap* tmO, uint64_t* bar, uint32_t item,
+                                          uint64_t policy) {
+    mbar_arrive_expect_tx(bar, kRItemBytes);
+    tma_load_2d_hint(slot, tmE, bar, 0, (int32_t)(item * 32), policy);
+    tma_load_2d_hint(slot + kRHalfBytes, tmO, bar, 0, (int32_t)(item * 32), policy);
+}
+
+// MODE 0: amax partials (one per CTA).  MODE 1: quantize.
 template <int G, int MODE>
-__global__ void __launch_bounds__(kTmaThreads, 1)
-    tma_unit_kernel(const __grid_constant__ CUtensorMap tmX, const UnitParams p,
-                    const TmaParams t, int* status) {
-    using S = TmaShape<G>;
-    constexpr int E = S::E;
-    constexpr int NCT = UnitShape<G>::NCT;
-    constexpr int SUBS = S::SUBS;
+__global__ void __launch_bounds__(kRThreads, 1)
+    row_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmO,
+               const UnitParams p, const RowParams t, int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRRingBytes);
     __shared__ float red[32];
     __shared__ float s_gsf;
     __shared__ float inv_tab[128];
     __shared__ int s_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = lane & 1;
     if (threadIdx.x == 0) s_abort = 0;
     if (lane == 0)
-        for (int s = 0; s < kSlots; ++s) mbar_init(&full[warp * kSlots + s], 1);
+        for (int s = 0; s < kRSlots; ++s) mbar_init(&full[warp * kRSlots + s], 1);
     fence_barrier_init();
     __syncthreads();
     griddep_wait();
@@ -470,96 +632,65 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
 
     float gsf = 0.0f;
     if constexpr (MODE == 1) {
-        gsf = encode_prologue<kTmaThreads>(p, red, &s_gsf, inv_tab);
-        // scale bytes of the padding rows (up to the next multiple of 128) are zero
-        const int64_t pad_rows = (p.rows + 127) / 128 * 128 - p.rows;
-        for (int64_t i = (int64_t)blockIdx.x * kTmaThreads + threadIdx.x; i < pad_rows * p.cgroups;
-             i += (int64_t)gridDim.x * kTmaThreads) {
-            const int64_t row = p.rows + i / p.cgroups, cg = i % p.cgroups;
-            const int64_t off = (((row >> 7) * p.cgroups + cg) << 9) + ((row & 31) << 4) +
-                                (((row >> 5) & 3) << 2);
-            *reinterpret_cast<uint32_t*>(p.sf + off) = 0u;
-        }
+        gsf = encode_prologue<kRThreads>(p, red, &s_gsf, inv_tab);
+        zero_padding_scales<kRThreads>(p);
     }
 
     const uint64_t policy = MODE == 0 ? l2_policy_evict_last() : l2_policy_evict_first();
-    const uint32_t stride = gridDim.x * kTmaWarps;
-    uint8_t* ring = smem + warp * kSlots * S::ITEM_BYTES;
-    uint64_t* bars = full + warp * kSlots;
-    const uint32_t first = blockIdx.x * kTmaWarps + warp;
-    if (lane == 0) {
-        for (int s = 0; s < kSlots; ++s) {
+    const uint32_t stride = gridDim.x * kRWarps;
+    uint8_t* ring = smem + warp * kRSlots * kRItemBytes;
+    uint64_t* bars = full + warp * kRSlots;
+    const uint32_t first = blockIdx.x * kRWarps + warp;
+    if (lane == 0)
+        for (int s = 0; s < kRSlots; ++s) {
             const uint32_t it = first + s * stride;
-            if (it < t.n_items) {
-                mbar_arrive_expect_tx(&bars[s], S::ITEM_BYTES);
-                tma_load_2d_hint(ring + s * S::ITEM_BYTES, &tmX, &bars[s], 0,
-                                 (int32_t)(it * kItemRows), policy);
-            }
+            if (it < t.n_items) load_item(ring + s * kRItemBytes, &tmE, &tmO, &bars[s], it, policy);
         }
-    }
 
-    const int pair = lane >> 1;
-    uint32_t tmax = 0u;       // packed bf16 maxima (G < 32)
-    float fmax_rot = 0.0f;    // pre-scale rotated maximum (G >= 32)
+    uint32_t tmax = 0u;       // packed bf16 maxima (G = 0)
+    float fmax_rot = 0.0f;    // pre-scale rotated maximum (G > 0)
     uint32_t k = 0;
     for (uint32_t item = first; item < t.n_items; item += stride, ++k) {
-        const int s = (int)(k % kSlots);
-        if (!mbar_wait_bounded(&bars[s], (k / kSlots) & 1u, &s_abort, status, kTmaWaitBudgetNs))
+        const int s = (int)(k % kRSlots);
+        if (!mbar_wait_bounded(&bars[s], (k / kRSlots) & 1u, &s_abort, status, kTmaWaitBudgetNs))
             break;
-        const uint8_t* slot = ring + s * S::ITEM_BYTES;
-        uint4 w[SUBS][NCT];
-#pragma unroll
-        for (int sub = 0; sub < SUBS; ++sub) {
-            const int m = item_unit<E>(pair, sub);
-#pragma unroll
-            for (int i = 0; i < NCT; ++i) {
-                const int j = 2 * i + h;                            // chunk of the unit
-                const int fr = (E == 128) ? 2 * m + (j >> 3) : m;   // flat row of the item
-                const int pos = (j & 7) ^ (fr & 7);
-                w[sub][i] = *reinterpret_cast<const uint4*>(slot + fr * 128 + pos * 16);
-            }
-        }
+        uint8_t* slot = ring + s * kRItemBytes;
+        uint4 w[16];
+        load_unit(slot, lane, w);
         __syncwarp();
         if (lane == 0) {
-            const uint32_t nxt = item + kSlots * stride;
+            const uint32_t nxt = item + kRSlots * stride;
             if (nxt < t.n_items) {
                 fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&bars[s], S::ITEM_BYTES);
-                tma_load_2d_hint(ring + s * S::ITEM_BYTES, &tmX, &bars[s], 0,
-                                 (int32_t)(nxt * kItemRows), policy);
+                load_item(slot, &tmE, &tmO, &bars[s], nxt, policy);
             }
         }
-#pragma unroll
-        for (int sub = 0; sub < SUBS; ++sub) {
-            const uint32_t unit = item * S::UPI + item_unit<E>(pair, sub);
-            const bool active = unit < t.total_units;
-            const uint32_t row = fast_div(unit, t.upr_div);
-            const int64_t e0 = (int64_t)(unit - row * t.upr) * E;
-            if constexpr (MODE == 0 && G >= 32) {
-                fmax_rot = rotate_amax<G>(w[sub], h, fmax_rot);
-            } else if constexpr (MODE == 0) {
-                if constexpr (G > 0) rotate_unit<G>(w[sub], h, p.hscale);
-#pragma unroll
-                for (int i = 0; i < NCT; ++i) tmax = absmax2_bf16(tmax, absmax_word4(w[sub][i]));
-            } else {
-                if constexpr (G > 0) rotate_unit<G>(w[sub], h, p.hscale);
-                encode_unit<G>(w[sub], h, gsf, inv_tab, p, (int64_t)row, e0, E, active, active);
+        // units past the end were zero-filled by the copy: they add nothing to the amax
+        if constexpr (MODE == 0) {
+            unit_amax<G>(w, tmax, fmax_rot);
+        } else {
+            const uint32_t unit = item * 32 + lane;
+            if (unit < t.total_units) {
+                const uint32_t row = fast_div(unit, t.upr_div);
+                float r[128];
+                unit_values<G>(w, p.hscale, r);
+                encode_unit128(r, gsf, inv_tab, p, (int64_t)row, (int64_t)(unit - row * t.upr) * 128);
             }
         }
     }
     if constexpr (MODE == 0) {
-        const float mine = G >= 32 ? rotated_amax_bf16(fmax_rot, p.hscale) : absmax_of_pair(tmax);
+        const float mine = G > 0 ? rotated_amax_bf16(fmax_rot, p.hscale) : absmax_of_pair(tmax);
         const float mx = block_max(mine, red);
         if (threadIdx.x == 0) p.partials_out[blockIdx.x] = mx;
     }
     // after a timeout, let this warp's loads still in flight land before the CTA exits
     if (s_abort && lane == 0) {
         volatile int no_abort = 0;
-        for (uint32_t s = 0; s < (uint32_t)kSlots; ++s) {
+        for (uint32_t s = 0; s < (uint32_t)kRSlots; ++s) {
             const uint32_t kk = k + s;
             const uint64_t it = first + (uint64_t)kk * stride;
             if (it < t.n_items)
-                mbar_wait_bounded(&bars[kk % kSlots], (kk / kSlots) & 1u, &no_abort, nullptr,
+                mbar_wait_bounded(&bars[kk % kRSlots], (kk / kRSlots) & 1u, &no_abort, nullptr,
                                   100000000ull);
         }
     }
@@ -567,95 +698,82 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Single pass for a dynamic scale when the whole call fits in shared memory at once
-// (every warp's items fit its three ring slots; 14.5 M values on 148 SMs -- a 4096 x
-// 1024 tile is 4.2 M).  Each warp loads its items once, rotates them in place in shared
-// memory while taking the amax, the CTAs meet at a grid barrier (cooperative launch, so
-// all of them are resident; the wait is bounded), and every warp then encodes its items
-// from shared memory with the global scale: one HBM read and one rotation instead of two.
-// The arithmetic is the two-pass kernels' own, so the results are identical.
+// (every warp's items fit its kRSlots ring slots: 148 x 12 x 2 items of 4096 values,
+// 14.5 M values on 148 SMs -- a 4096 x 1024 tile is 4.2 M).  Each warp loads its items
+// once, rotates them in place in shared memory while taking the amax, the CTAs meet at a
+// grid barrier (cooperative launch, so all of them are resident; the wait is bounded),
+// and every warp then encodes its items from shared memory with the global scale: one
+// HBM read and one rotation instead of two.  The arithmetic is the two-pass kernels'
+// own, so the results are identical.
 // ---------------------------------------------------------------------------
 
 template <int G>
-__global__ void __launch_bounds__(kTmaThreads, 1)
-    single_pass_kernel(const __grid_constant__ CUtensorMap tmX, const UnitParams p,
-                       const TmaParams t, float* partials, unsigned int* arrive, int* status) {
-    using S = TmaShape<G>;
-    constexpr int E = S::E;
-    constexpr int NCT = UnitShape<G>::NCT;
-    constexpr int SUBS = S::SUBS;
+__global__ void __launch_bounds__(kRThreads, 1)
+    row_single_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmO,
+                      const UnitParams p, const RowParams t, float* partials,
+                      unsigned int* arrive, int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRRingBytes);
     __shared__ float red[32];
     __shared__ float s_gsf;
     __shared__ float inv_tab[128];
     __shared__ int s_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = lane & 1;
-    const int pair = lane >> 1;
     if (threadIdx.x == 0) s_abort = 0;
     if (lane == 0)
-        for (int s = 0; s < kSlots; ++s) mbar_init(&full[warp * kSlots + s], 1);
+        for (int s = 0; s < kRSlots; ++s) mbar_init(&full[warp * kRSlots + s], 1);
     fence_barrier_init();
     __syncthreads();
 
-    const uint32_t stride = gridDim.x * kTmaWarps;
-    const uint32_t first = blockIdx.x * kTmaWarps + warp;
-    uint8_t* ring = smem + warp * kSlots * S::ITEM_BYTES;
-    uint64_t* bars = full + warp * kSlots;
+    const uint32_t stride = gridDim.x * kRWarps;
+    const uint32_t first = blockIdx.x * kRWarps + warp;
+    uint8_t* ring = smem + warp * kRSlots * kRItemBytes;
+    uint64_t* bars = full + warp * kRSlots;
     if (lane == 0)
-        for (int k = 0; k < kSlots; ++k) {
-            const uint32_t it = first + k * stride;
-            if (it < t.n_items) {
-                mbar_arrive_expect_tx(&bars[k], S::ITEM_BYTES);
-                tma_load_2d(ring + k * S::ITEM_BYTES, &tmX, &bars[k], 0, (int32_t)(it * kItemRows));
-            }
+        for (int s = 0; s < kRSlots; ++s) {
+            const uint32_t it = first + s * stride;
+            if (it < t.n_items)
+                load_item(ring + s * kRItemBytes, &tmE, &tmO, &bars[s], it, l2_policy_evict_first());
         }
-
-    // the swizzled position of chunk i of sub-unit `sub` of this lane in an item
-    auto chunk_ptr = [&](uint8_t* slot, int sub, int i) -> uint4* {
-        const int m = item_unit<E>(pair, sub);
-        const int j = 2 * i + h;
-        const int fr = (E == 128) ? 2 * m + (j >> 3) : m;
-        return reinterpret_cast<uint4*>(slot + fr * 128 + (((j & 7) ^ (fr & 7)) << 4));
-    };
 
     // pass over the own items: rotate in place, amax of the rotated values
     uint32_t tmax = 0u;
     bool ok = true;
-    for (int k = 0; k < kSlots; ++k) {
-        const uint32_t item = first + k * stride;
+    for (int s = 0; s < kRSlots; ++s) {
+        const uint32_t item = first + s * stride;
         if (item >= t.n_items) break;
-        if (!mbar_wait_bounded(&bars[k], 0u, &s_abort, status, kTmaWaitBudgetNs)) {
+        if (!mbar_wait_bounded(&bars[s], 0u, &s_abort, status, kTmaWaitBudgetNs)) {
             ok = false;
             break;
         }
-        uint8_t* slot = ring + k * S::ITEM_BYTES;
+        uint8_t* slot = ring + s * kRItemBytes;
+        uint4 w[16];
+        load_unit(slot, lane, w);
+        if constexpr (G > 0) {
+            float r[128];
+            unit_values<G>(w, p.hscale, r);
 #pragma unroll
-        for (int sub = 0; sub < SUBS; ++sub) {
-            uint4 w[NCT];
-#pragma unroll
-            for (int i = 0; i < NCT; ++i) w[i] = *chunk_ptr(slot, sub, i);
-            if constexpr (G > 0) {
-                rotate_unit<G>(w, h, p.hscale);
-#pragma unroll
-                for (int i = 0; i < NCT; ++i) *chunk_ptr(slot, sub, i) = w[i];
+            for (int c = 0; c < 16; ++c) {
+                w[c] = make_uint4(pack_bf16_pair(r[8 * c], r[8 * c + 1]),
+                                  pack_bf16_pair(r[8 * c + 2], r[8 * c + 3]),
+                                  pack_bf16_pair(r[8 * c + 4], r[8 * c + 5]),
+                                  pack_bf16_pair(r[8 * c + 6], r[8 * c + 7]));
+                *reinterpret_cast<uint4*>(slot + unit_chunk_off(lane, c)) = w[c];
             }
-            // units past the end hold the zeros the copy filled in: they add nothing
+        }
+        // units past the end hold the zeros the copy filled in: they add nothing
 #pragma unroll
-            for (int i = 0; i < NCT; ++i) tmax = absmax2_bf16(tmax, absmax_word4(w[i]));
-        }
+        for (int c = 0; c < 16; ++c) tmax = absmax2_bf16(tmax, absmax_word4(w[c]));
     }
-    if (!ok) {
+    if (!ok && lane == 0) {
         // let this warp's other loads land before the CTA can leave
-        if (lane == 0) {
-            volatile int no_abort = 0;
-            for (int k = 0; k < kSlots; ++k)
-                if (first + k * stride < t.n_items)
-                    mbar_wait_bounded(&bars[k], 0u, &no_abort, nullptr, 100000000ull);
-        }
+        volatile int no_abort = 0;
+        for (int s = 0; s < kRSlots; ++s)
+            if (first + s * stride < t.n_items)
+                mbar_wait_bounded(&bars[s], 0u, &no_abort, nullptr, 100000000ull);
     }
 
     // grid-wide amax: per-CTA partials, then a bounded barrier on the arrival count
@@ -679,7 +797,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
 
     // the global scale from every CTA's partial (read past L1), then the encode table
     float mm = 0.0f;
-    for (int i = threadIdx.x; i < (int)gridDim.x; i += kTmaThreads) mm = fmaxf(mm, __ldcg(partials + i));
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += kRThreads) mm = fmaxf(mm, __ldcg(partials + i));
     mm = block_max(mm, red);
     if (threadIdx.x == 0) s_gsf = __fdiv_rn(kFp4E4m3Range, fmaxf(mm, kAmaxFloor));
     __syncthreads();
@@ -692,74 +810,107 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         const float sv = f32_from_e4m3(threadIdx.x);
         inv_tab[threadIdx.x] = (threadIdx.x == 0 || threadIdx.x == 127) ? 0.0f : __fdiv_rn(gsf, sv);
     }
-    // scale bytes of the padding rows (up to the next multiple of 128) are zero
-    const int64_t pad_rows = (p.rows + 127) / 128 * 128 - p.rows;
-    for (int64_t i = (int64_t)blockIdx.x * kTmaThreads + threadIdx.x; i < pad_rows * p.cgroups;
-         i += (int64_t)gridDim.x * kTmaThreads) {
-        const int64_t row = p.rows + i / p.cgroups, cg = i % p.cgroups;
-        const int64_t off = (((row >> 7) * p.cgroups + cg) << 9) + ((row & 31) << 4) +
-                            (((row >> 5) & 3) << 2);
-        *reinterpret_cast<uint32_t*>(p.sf + off) = 0u;
-    }
+    zero_padding_scales<kRThreads>(p);
     __syncthreads();
 
     // encode the own items from shared memory
-    for (int k = 0; k < kSlots; ++k) {
-        const uint32_t item = first + k * stride;
+    for (int s = 0; s < kRSlots; ++s) {
+        const uint32_t item = first + s * stride;
         if (item >= t.n_items) break;
-        uint8_t* slot = ring + k * S::ITEM_BYTES;
-#pragma unroll
-        for (int sub = 0; sub < SUBS; ++sub) {
-            uint4 w[NCT];
-#pragma unroll
-            for (int i = 0; i < NCT; ++i) w[i] = *chunk_ptr(slot, sub, i);
-            const uint32_t unit = item * S::UPI + item_unit<E>(pair, sub);
-            const bool active = unit < t.total_units;
-            const uint32_t row = fast_div(unit, t.upr_div);
-            const int64_t e0 = (int64_t)(unit - row * t.upr) * E;
-            encode_unit<G>(w, h, gsf, inv_tab, p, (int64_t)row, e0, E, active, active);
-        }
+        const uint32_t unit = item * 32 + lane;
+        if (unit >= t.total_units) continue;
+        uint4 w[16];
+        load_unit(ring + s * kRItemBytes, lane, w);
+        float r[128];
+        unit_values<0>(w, 1.0f, r);
+        const uint32_t row = fast_div(unit, t.upr_div);
+        encode_unit128(r, gsf, inv_tab, p, (int64_t)row, (int64_t)(unit - row * t.upr) * 128);
     }
 }
 
+template <typename Kernel>
+bool set_smem_once(Kernel* k, std::atomic<int> (&flags)[64], int device, int bytes) {
+    if (flags[device].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return false;
+    flags[device].store(1, std::memory_order_release);
+    return true;
+}
+
 template <int G>
-nvfp4_status launch_single_pass(const CUtensorMap& map, const UnitParams& p, const TmaParams& t,
-                                int grid, float* partials, int device, int* status,
-                                cudaStream_t stream) {
-    constexpr int smem = TmaShape<G>::SMEM;
+nvfp4_status launch_row_single(const CUtensorMap& mE, const CUtensorMap& mO, const UnitParams& p,
+                               const RowParams& t, int grid, float* partials, int device,
+                               int* status, cudaStream_t stream) {
     static std::atomic<int> attr_set[64];
     if (device < 0 || device >= 64) return NVFP4_ERR_DEVICE;
-    if (!attr_set[device].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(single_pass_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem) != cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        attr_set[device].store(1, std::memory_order_release);
-    }
+    if (!set_smem_once(row_single_kernel<G>, attr_set, device, kRSmem)) return NVFP4_ERR_CUDA;
     // the arrival counter lives in the last word of the caller's 4 KiB workspace
     unsigned int* arrive = reinterpret_cast<unsigned int*>(partials) + (kMaxPartials - 1);
     if (cudaMemsetAsync(arrive, 0, sizeof(unsigned int), stream) != cudaSuccess)
         return NVFP4_ERR_CUDA;
-    const CUtensorMap* mp = &map;
-    void* args[] = {const_cast<CUtensorMap*>(mp), const_cast<UnitParams*>(&p),
-                    const_cast<TmaParams*>(&t), &partials, &arrive, &status};
-    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(single_pass_kernel<G>), dim3(grid),
-                                    dim3(kTmaThreads), args, smem, stream) != cudaSuccess)
+    void* args[] = {const_cast<CUtensorMap*>(&mE), const_cast<CUtensorMap*>(&mO),
+                    const_cast<UnitParams*>(&p), const_cast<RowParams*>(&t), &partials, &arrive,
+                    &status};
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(row_single_kernel<G>), dim3(grid),
+                                    dim3(kRThreads), args, kRSmem, stream) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
 }
 
-nvfp4_status dispatch_single_pass(int g, const CUtensorMap& map, const UnitParams& p,
-                                  const TmaParams& t, int grid, float* partials, int device,
-                                  int* status, cudaStream_t stream) {
+nvfp4_status dispatch_row_single(int g, const CUtensorMap& mE, const CUtensorMap& mO,
+                                 const UnitParams& p, const RowParams& t, int grid,
+                                 float* partials, int device, int* status, cudaStream_t stream) {
     switch (g) {
-        case 0: return launch_single_pass<0>(map, p, t, grid, partials, device, status, stream);
-        case 16: return launch_single_pass<16>(map, p, t, grid, partials, device, status, stream);
-        case 32: return launch_single_pass<32>(map, p, t, grid, partials, device, status, stream);
-        case 64: return launch_single_pass<64>(map, p, t, grid, partials, device, status, stream);
-        case 128: return launch_single_pass<128>(map, p, t, grid, partials, device, status, stream);
+        case 0: return launch_row_single<0>(mE, mO, p, t, grid, partials, device, status, stream);
+        case 16: return launch_row_single<16>(mE, mO, p, t, grid, partials, device, status, stream);
+        case 32: return launch_row_single<32>(mE, mO, p, t, grid, partials, device, status, stream);
+        case 64: return launch_row_single<64>(mE, mO, p, t, grid, partials, device, status, stream);
+        case 128: return launch_row_single<128>(mE, mO, p, t, grid, partials, device, status, stream);
         default: break;
     }
     return NVFP4_ERR_INVALID_ARG;
+}
+
+template <int G, int MODE>
+nvfp4_status launch_row(const CUtensorMap& mE, const CUtensorMap& mO, const UnitParams& p,
+                        const RowParams& t, int grid, int device, int* status, cudaStream_t stream) {
+    static std::atomic<int> attr_set[64];
+    if (device < 0 || device >= 64) return NVFP4_ERR_DEVICE;
+    if (!set_smem_once(row_kernel<G, MODE>, attr_set, device, kRSmem)) return NVFP4_ERR_CUDA;
+    if (launch_pdl(row_kernel<G, MODE>, (unsigned)grid, kRThreads, kRSmem, stream, mE, mO, p, t,
+                   status) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
+
+template <int MODE>
+nvfp4_status dispatch_row(int g, const CUtensorMap& mE, const CUtensorMap& mO, const UnitParams& p,
+                          const RowParams& t, int grid, int device, int* status, cudaStream_t stream) {
+    switch (g) {
+        case 0: return launch_row<0, MODE>(mE, mO, p, t, grid, device, status, stream);
+        case 16: return launch_row<16, MODE>(mE, mO, p, t, grid, device, status, stream);
+        case 32: return launch_row<32, MODE>(mE, mO, p, t, grid, device, status, stream);
+        case 64: return launch_row<64, MODE>(mE, mO, p, t, grid, device, status, stream);
+        case 128: return launch_row<128, MODE>(mE, mO, p, t, grid, device, status, stream);
+        default: break;
+    }
+    return NVFP4_ERR_INVALID_ARG;
+}
+
+// One half of every 128-value unit of x: [n_units, 64] bf16 rows 256 bytes apart, based at
+// x (first halves) or x + 128 bytes (second halves), with a [32, 64] box and the 128-byte
+// swizzle.
+bool make_half_map(CUtensorMap* map, const void* base, int64_t n_units) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {64, (cuuint64_t)n_units};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 template <int G, int MODE>
@@ -779,52 +930,6 @@ nvfp4_status dispatch(int g, const UnitParams& p, int grid, cudaStream_t stream)
         default: break;
     }
     return NVFP4_ERR_INVALID_ARG;
-}
-
-template <int G, int MODE>
-nvfp4_status launch_tma_unit(const CUtensorMap& map, const UnitParams& p, const TmaParams& t,
-                             int grid, int device, int* status, cudaStream_t stream) {
-    constexpr int smem = TmaShape<G>::SMEM;
-    static std::atomic<int> attr_set[64];
-    if (device < 0 || device >= 64) return NVFP4_ERR_DEVICE;
-    if (!attr_set[device].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(tma_unit_kernel<G, MODE>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        attr_set[device].store(1, std::memory_order_release);
-    }
-    if (launch_pdl(tma_unit_kernel<G, MODE>, (unsigned)grid, kTmaThreads, smem, stream, map, p, t,
-                   status) != cudaSuccess)
-        return NVFP4_ERR_CUDA;
-    return NVFP4_OK;
-}
-
-template <int MODE>
-nvfp4_status dispatch_tma(int g, const CUtensorMap& map, const UnitParams& p, const TmaParams& t,
-                          int grid, int device, int* status, cudaStream_t stream) {
-    switch (g) {
-        case 0: return launch_tma_unit<0, MODE>(map, p, t, grid, device, status, stream);
-        case 16: return launch_tma_unit<16, MODE>(map, p, t, grid, device, status, stream);
-        case 32: return launch_tma_unit<32, MODE>(map, p, t, grid, device, status, stream);
-        case 64: return launch_tma_unit<64, MODE>(map, p, t, grid, device, status, stream);
-        case 128: return launch_tma_unit<128, MODE>(map, p, t, grid, device, status, stream);
-        default: break;
-    }
-    return NVFP4_ERR_INVALID_ARG;
-}
-
-// x as [rows*K/64, 64] bf16 with a [BR, 64] box and the 128-byte swizzle.
-bool make_flat_map(CUtensorMap* map, const void* x, int64_t flat_rows, int box_rows) {
-    auto enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {64, (cuuint64_t)flat_rows};
-    cuuint64_t strides[1] = {128};
-    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(x), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
 }
 
 int64_t unit_elems(int g) { return g == 128 ? 128 : 64; }
@@ -861,38 +966,39 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
     p.gsf_w = gsf_w;
     p.alpha_out = alpha_out;
 
-    const int64_t flat_rows = rows * K / 64;
-    if (K % 64 == 0 && flat_rows < (int64_t(1) << 31) - 256) {
+    const int64_t n_units = rows * (K / 128);
+    if (K % 128 == 0 && n_units < (int64_t(1) << 31) - 64) {
         int* status = nullptr;
         if ((st = status_word(&status)) != NVFP4_OK) return st;
-        CUtensorMap map;
-        if (!make_flat_map(&map, x, flat_rows, kItemRows)) return NVFP4_ERR_CUDA;
-        const int upi = group == 128 ? 16 : 32;
-        p.total_units = rows * p.upr;
-        TmaParams t;
-        t.total_units = (uint32_t)p.total_units;
-        t.n_items = (uint32_t)((p.total_units + upi - 1) / upi);
-        t.upr = (uint32_t)p.upr;
+        CUtensorMap mE, mO;
+        if (!make_half_map(&mE, x, n_units) ||
+            !make_half_map(&mO, static_cast<const uint8_t*>(x) + 128, n_units))
+            return NVFP4_ERR_CUDA;
+        p.total_units = n_units;
+        RowParams t;
+        t.total_units = (uint32_t)n_units;
+        t.n_items = (uint32_t)((n_units + 31) / 32);
+        t.upr = (uint32_t)(K / 128);
         t.upr_div = make_fastdiv(t.upr);
-        // dynamic scale that fits on chip: one pass, every warp holding at most kSlots items
-        const int64_t per_cta = (int64_t)kTmaWarps * kSlots;
-        if (gsf_in == nullptr && (int64_t)t.n_items <= (int64_t)dev.sms * per_cta) {
+        // dynamic scale that fits on chip: one pass, every warp holding at most kRSlots items
+        if (gsf_in == nullptr && (int64_t)t.n_items <= (int64_t)dev.sms * kRWarps * kRSlots) {
             // as many CTAs as give every warp one item, up to one per SM
-            const int64_t g1 = ((int64_t)t.n_items + kTmaWarps - 1) / kTmaWarps;
-            return dispatch_single_pass(group, map, p, t, (int)(g1 < dev.sms ? (g1 > 0 ? g1 : 1) : dev.sms),
-                                        partials, dev.device, status, stream);
+            const int64_t g1 = ((int64_t)t.n_items + kRWarps - 1) / kRWarps;
+            return dispatch_row_single(group, mE, mO, p, t,
+                                       (int)(g1 < dev.sms ? (g1 > 0 ? g1 : 1) : dev.sms), partials,
+                                       dev.device, status, stream);
         }
-        const int64_t need = (t.n_items + kTmaWarps - 1) / kTmaWarps;
+        const int64_t need = ((int64_t)t.n_items + kRWarps - 1) / kRWarps;
         const int grid = (int)(need < dev.sms ? (need > 0 ? need : 1) : dev.sms);
         if (gsf_in == nullptr) {
             UnitParams a = p;
             a.partials_out = partials;
-            st = dispatch_tma<0>(group, map, a, t, grid, dev.device, status, stream);
+            st = dispatch_row<0>(group, mE, mO, a, t, grid, dev.device, status, stream);
             if (st != NVFP4_OK) return st;
             p.partials = partials;
             p.n_partials = grid;
         }
-        return dispatch_tma<1>(group, map, p, t, grid, dev.device, status, stream);
+        return dispatch_row<1>(group, mE, mO, p, t, grid, dev.device, status, stream);
     }
 
     if (gsf_in == nullptr) {

@@ -173,14 +173,23 @@ def test_dynamic_two_pass_rotated(oracle, group):
 
 
 @pytest.mark.parametrize("sign", [1.0, -1.0])
-@pytest.mark.parametrize("R,K", [(3, 96), (257, 160)])
-def test_dynamic_amax_last_stage_branch(oracle, sign, R, K):
+@pytest.mark.parametrize("group,R,K", [(32, 3, 96), (32, 257, 160),
+                                       (16, 3, 256), (32, 130, 256), (64, 3, 256), (128, 257, 256)])
+def test_dynamic_amax_last_stage_branch(oracle, sign, group, R, K):
     """The largest rotated value comes out of the last stage's sum (sign +1) or its
-    difference (sign -1): g = 32 over [1, 0 x 15, sign, 0 x 15] gives halves of all ones and
-    all `sign`, so a + b or a - b is 2 and the other is 0.  K % 64 != 0 keeps the plain-load
-    kernels (amax pass, then encode pass)."""
-    g = torch.Generator().manual_seed(int(K + 10 * sign))
+    difference (sign -1): a g-group [1, 0 x (g/2 - 1), sign, 0 x (g/2 - 1)] gives halves of
+    all ones and all `sign` before the last stage, so a + b or a - b is 2 and the other is
+    0.  K % 128 != 0 runs the lane-pair kernels, K % 128 == 0 the one-thread-per-unit
+    kernels; both take max(|a| + |b|) before the last stage in the amax pass."""
+    g = torch.Generator().manual_seed(int(K + 10 * sign + group))
     x = torch.randn(R, K, generator=g) * 1e-3
-    x[1, 32] = 1.0
-    x[1, 48] = sign
-    check(oracle, x.to(torch.bfloat16), 32, None)
+    x[1, group] = 1.0
+    x[1, group + group // 2] = sign
+    xb = x.to(torch.bfloat16)
+    check(oracle, xb, group, None)
+    # the same rows repeated past the single-pass capacity (14.55 M values on 148 SMs):
+    # the two-pass route, amax pass then encode pass
+    if K % 128 == 0:
+        rows = 14_700_000 // K + 1
+        big = xb.repeat(rows // R + 1, 1)[:rows].contiguous()
+        check(oracle, big, group, None)
