@@ -142,6 +142,49 @@ def time_each(fn, reps: int, flush: torch.Tensor | None = None, warmup: int = 3)
     return sum(e0.elapsed_time(e1) for e0, e1 in pairs) / reps
 
 
+def time_graph(fn, reps: int, flush: torch.Tensor | None = None) -> float | None:
+    """Mean ms of one call inside a CUDA graph of `reps` calls (each after a write of
+    `flush`, larger than L2, when given), minus the same graph without the calls: the
+    device time without the host's per-call launch cost.  None if the call cannot be
+    captured."""
+    def capture(with_call):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            fn()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(reps):
+                    if flush is not None:
+                        flush.fill_(1.0)
+                    if with_call:
+                        fn()
+        torch.cuda.synchronize()
+        return g
+
+    try:
+        g1, g0 = capture(True), (capture(False) if flush is not None else None)
+    except Exception:
+        torch.cuda.synchronize()
+        return None
+
+    def run(g):
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    t1 = min(run(g1) for _ in range(3))
+    t0 = min(run(g0) for _ in range(3)) if g0 is not None else 0.0
+    del g1, g0
+    return (t1 - t0) / reps
+
+
 def l2_flush_buffer(dev):
     return torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB
 
@@ -430,10 +473,13 @@ def leg_tiny(dev, pk, l2):
     scale, no rotation) through nvfp4_linear: launch-bound, timed as back-to-back calls."""
     lin = W.tiny(dev)
     ly = Layer(lin, dev, group=0)
-    ms = time_loop(lambda: ly.linear(True), 200, 10)
+    ms_eager = time_loop(lambda: ly.linear(True), 200, 10)
+    ms_graph = time_graph(lambda: ly.linear(True), 50)
+    ms = ms_graph if ms_graph is not None else ms_eager
     f = ly.flops()
     return {"workload": "tiny W4A4 linear 128 x 256 x 256, dynamic scale, bias",
-            "us": ms * 1e3, "TFLOP/s": f / (ms * 1e-3) / 1e12,
+            "us": ms * 1e3, "TFLOP/s": f / (ms * 1e-3) / 1e12, "eager_us": ms_eager * 1e3,
+            "timing": "CUDA graph of 50 calls back to back" if ms_graph is not None else "eager",
             "launches": quantizer_launches(128, 256, 0, True) + 1,
             "note": "launch-bound: 16.8 MFLOP per call"}
 
@@ -514,17 +560,22 @@ def leg_linear_m_sweep(dev, pk, l2):
     for M in W.M_SWEEP:
         lin = W.m_sweep(M, dev)
         ly = Layer(lin, dev, group=0)
-        ms = time_each(lambda: ly.linear(True), 10, flush)
+        ms_eager = time_each(lambda: ly.linear(True), 10, flush)
+        ms_graph = time_graph(lambda: ly.linear(True), 10, flush)
+        ms = ms_graph if ms_graph is not None else ms_eager
         tot, qb, gb = linear_bytes(M, 5120, 5120, True, l2)
         tf = ly.flops() / (ms * 1e-3) / 1e12
         gbps = tot / (ms * 1e-3) / 1e9
         pts.append({"M": M, "us": ms * 1e3, "TFLOP/s": tf, "frac_of_fp4_peak": tf / pk["fp4"],
-                    "GBps": gbps, "frac_of_hbm": gbps / pk["hbm"],
+                    "GBps": gbps, "frac_of_hbm": gbps / pk["hbm"], "eager_us": ms_eager * 1e3,
+                    "timing": "graph" if ms_graph is not None else "eager",
                     "launches": quantizer_launches(M, 5120, 0, True) + 1})
         del ly, lin
     del flush
     return {"workload": "nvfp4_linear_prepared, N = K = 5120, dynamic scale, no bias, L2 "
-                        "flushed before each call", "points": pts}
+                        "flushed before each call; us from a CUDA graph of flush + call pairs "
+                        "minus the flushes alone (eager_us: events around each eager call)",
+            "points": pts}
 
 
 def leg_gemm_m_sweep(dev, pk, l2):
@@ -551,17 +602,21 @@ def leg_gemm_m_sweep(dev, pk, l2):
     for M in W.M_SWEEP:
         xp, xsf = operand(M)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        ms = time_each(lambda: nv.nvfp4_gemm_prepared(xp, xsf, wp, wsf, alpha, None, M, N, K,
-                                                      out=y), 10, flush)
+        call = lambda: nv.nvfp4_gemm_prepared(xp, xsf, wp, wsf, alpha, None, M, N, K, out=y)
+        ms_eager = time_each(call, 10, flush)
+        ms_graph = time_graph(call, 10, flush)
+        ms = ms_graph if ms_graph is not None else ms_eager
         tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
         gb = (N * K * 0.5625 + M * K * 0.5625 + 2.0 * M * N) / (ms * 1e-3) / 1e9
         points.append({"M": M, "us": ms * 1e3, "TFLOP/s": tf,
                        "frac_of_fp4_peak": tf / pk["fp4"], "GBps": gb,
-                       "frac_of_hbm": gb / pk["hbm"]})
+                       "frac_of_hbm": gb / pk["hbm"], "eager_us": ms_eager * 1e3,
+                       "timing": "graph" if ms_graph is not None else "eager"})
         del xp, xsf, y
     del flush
     return {"workload": "nvfp4_gemm_prepared, N = K = 5120, no bias, L2 flushed before each "
-                        "launch", "points": points}
+                        "launch; us from a CUDA graph of flush + call pairs minus the flushes "
+                        "alone (eager_us: events around each eager call)", "points": points}
 
 
 def leg_weight_pack(dev, pk, l2):

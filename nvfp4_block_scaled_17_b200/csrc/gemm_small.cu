@@ -1,4 +1,6 @@
-// gemm_small.cu -- the block-scaled FP4 GEMM for few activation rows (M <= 128).
+// gemm_small.cu -- the block-scaled FP4 GEMM for few activation rows (the kernel takes
+// M <= 128; nvfp4_gemm routes M <= 32 here, where it measured faster than the general
+// kernel's split-K build).
 //
 // Pages: "minimax_h3_nvfp4_decoder" -- nvfp4_linear_inference (mm_fp4 with alpha =
 // 1/(global_sf_x * global_sf_w), bf16 output, then the bias); the operation is the one

@@ -74,8 +74,10 @@ nvfp4_status launch_gemm_f32(const uint8_t* a, const uint8_t* sfa, const uint8_t
 // The GEMM for M <= kSmallMaxRows activation rows with the operands swapped
 // (y^T = W x^T: weight rows on the MMA's M, activation rows on its N), K split over a
 // thread-block cluster; same arguments and result as launch_gemm / launch_gemm_prepared
-// (sfb_prepared) / launch_gemm_f32 (f32_out, y is then float*).
-constexpr int64_t kSmallMaxRows = 128;
+// (sfb_prepared) / launch_gemm_f32 (f32_out, y is then float*).  The kernel takes up to
+// 128 rows; the dispatch uses it up to 32, where it measured faster than the general
+// kernel's split-K build (its reduction grows with M).
+constexpr int64_t kSmallMaxRows = 32;
 nvfp4_status launch_gemm_small(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                                const uint8_t* sfb, bool sfb_prepared, bool f32_out,
                                const float* alpha, const void* bias, void* y, int64_t M,

@@ -727,6 +727,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
         for (int s = 0; s < kRSlots; ++s) mbar_init(&full[warp * kRSlots + s], 1);
     fence_barrier_init();
     __syncthreads();
+    // a one-CTA call is launched with programmatic stream serialization (a cooperative
+    // grid is not): wait for the previous kernel before the first global access
+    griddep_wait();
+    griddep_launch_dependents();
 
     const uint32_t stride = gridDim.x * kRWarps;
     const uint32_t first = blockIdx.x * kRWarps + warp;
@@ -776,9 +780,12 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 mbar_wait_bounded(&bars[s], 0u, &no_abort, nullptr, 100000000ull);
     }
 
-    // grid-wide amax: per-CTA partials, then a bounded barrier on the arrival count
+    // grid-wide amax: per-CTA partials, then a bounded barrier on the arrival count (a
+    // one-CTA grid needs neither)
     const float m = block_max(absmax_of_pair(tmax), red);
-    if (threadIdx.x == 0) {
+    if (gridDim.x == 1) {
+        if (threadIdx.x == 0) s_gsf = m;
+    } else if (threadIdx.x == 0) {
         partials[blockIdx.x] = m;
         __threadfence();
         atomicAdd(arrive, 1u);
@@ -797,8 +804,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
 
     // the global scale from every CTA's partial (read past L1), then the encode table
     float mm = 0.0f;
-    for (int i = threadIdx.x; i < (int)gridDim.x; i += kRThreads) mm = fmaxf(mm, __ldcg(partials + i));
-    mm = block_max(mm, red);
+    if (gridDim.x == 1) {
+        mm = s_gsf;   // the block's own maximum, published above
+        __syncthreads();
+    } else {
+        for (int i = threadIdx.x; i < (int)gridDim.x; i += kRThreads) mm = fmaxf(mm, __ldcg(partials + i));
+        mm = block_max(mm, red);
+    }
     if (threadIdx.x == 0) s_gsf = __fdiv_rn(kFp4E4m3Range, fmaxf(mm, kAmaxFloor));
     __syncthreads();
     const float gsf = s_gsf;
@@ -846,6 +858,13 @@ nvfp4_status launch_row_single(const CUtensorMap& mE, const CUtensorMap& mO, con
     if (!set_smem_once(row_single_kernel<G>, attr_set, device, kRSmem)) return NVFP4_ERR_CUDA;
     // the arrival counter lives in the last word of the caller's 4 KiB workspace
     unsigned int* arrive = reinterpret_cast<unsigned int*>(partials) + (kMaxPartials - 1);
+    if (grid == 1) {
+        // one CTA: no grid barrier, so no counter to clear and no cooperative launch
+        if (launch_pdl(row_single_kernel<G>, 1u, kRThreads, kRSmem, stream, mE, mO, p, t, partials,
+                       arrive, status) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        return NVFP4_OK;
+    }
     if (cudaMemsetAsync(arrive, 0, sizeof(unsigned int), stream) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     void* args[] = {const_cast<CUtensorMap*>(&mE), const_cast<CUtensorMap*>(&mO),
@@ -982,8 +1001,11 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
         t.upr_div = make_fastdiv(t.upr);
         // dynamic scale that fits on chip: one pass, every warp holding at most kRSlots items
         if (gsf_in == nullptr && (int64_t)t.n_items <= (int64_t)dev.sms * kRWarps * kRSlots) {
-            // as many CTAs as give every warp one item, up to one per SM
-            const int64_t g1 = ((int64_t)t.n_items + kRWarps - 1) / kRWarps;
+            // one CTA when its slots hold the whole call (no grid barrier: an ordinary
+            // launch), else as many CTAs as give every warp one item, up to one per SM
+            const int64_t g1 = (int64_t)t.n_items <= kRWarps * kRSlots
+                                   ? 1
+                                   : ((int64_t)t.n_items + kRWarps - 1) / kRWarps;
             return dispatch_row_single(group, mE, mO, p, t,
                                        (int)(g1 < dev.sms ? (g1 > 0 ? g1 : 1) : dev.sms), partials,
                                        dev.device, status, stream);

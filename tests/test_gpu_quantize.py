@@ -18,13 +18,16 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def gpu_quantize(x: torch.Tensor, group: int, gsf):
+def gpu_quantize(x: torch.Tensor, group: int, gsf, ws_bytes=None):
+    """ws_bytes None: the binding's default workspace; otherwise a workspace of exactly
+    that many bytes."""
     R, K = x.shape
     packed = torch.full((R, K // 2), 0xAB, dtype=torch.uint8, device=DEV)     # garbage first
     sf = torch.full((nv.nvfp4_scale_bytes(R, K),), 0xAB, dtype=torch.uint8, device=DEV)
     gsf_out = torch.full((1,), -7.0, dtype=torch.float32, device=DEV)
     g_in = None if gsf is None else torch.tensor([gsf], dtype=torch.float32, device=DEV)
-    nv.nvfp4_quantize(x, group, g_in, out=(packed, sf, gsf_out))
+    ws = None if ws_bytes is None else torch.empty(ws_bytes, dtype=torch.uint8, device=DEV)
+    nv.nvfp4_quantize(x, group, g_in, out=(packed, sf, gsf_out), workspace=ws)
     torch.cuda.synchronize()
     return to_np(packed), to_np(sf), np.float32(gsf_out.item())
 
@@ -36,8 +39,8 @@ def oracle_quantize(oracle, x: torch.Tensor, group: int, gsf):
     return oracle.quantize(xu, gsf)
 
 
-def check(oracle, x, group, gsf):
-    p, s, g = gpu_quantize(x.to(DEV), group, gsf)
+def check(oracle, x, group, gsf, ws_bytes=None):
+    p, s, g = gpu_quantize(x.to(DEV), group, gsf, ws_bytes)
     op, os_, og = oracle_quantize(oracle, x, group, gsf)
     assert np.float32(og).view(np.uint32) == g.view(np.uint32), (og, g)
     assert np.array_equal(s, os_), f"scale bytes differ at {np.flatnonzero(s != os_)[:8]}"
@@ -161,12 +164,23 @@ def test_dynamic_single_pass_capacity_edge(oracle, group, rows):
     assert np.array_equal(to_np(p), op) and np.array_equal(to_np(sf), osf)
 
 
+@pytest.mark.parametrize("group", [0, 128])
+@pytest.mark.parametrize("rows", [1, 96, 97, 100])
+def test_dynamic_single_pass_one_cta_edge(oracle, group, rows):
+    """A dynamic call of at most 24 items of 32 units (96 x 1024: 768 units) runs the
+    single-pass kernel as one CTA, with no grid barrier; 97 rows need a 25th item and a
+    cooperative grid of CTAs.  Both bit for bit against the oracle."""
+    K = 1024
+    x = W.with_outliers((rows, K), 0.01, 20.0, W._gen(rows * 5 + group, "cpu"), "cpu")
+    check(oracle, x, group, None)
+
+
 @pytest.mark.parametrize("group", [16, 32, 64, 128])
 def test_dynamic_two_pass_rotated(oracle, group):
     """Past the single-pass capacity (16384 x 1024 = 16.8 M values) a dynamic call runs the
-    amax pass, then the encode pass.  With g >= 32 the amax pass stops before the last
-    butterfly stage, keeps max(|a| + |b|) of its operand pairs, and scales and rounds that
-    maximum once; the global scale must still equal the oracle's bit for bit."""
+    amax pass, then the encode pass.  The amax pass stops before the last butterfly stage,
+    keeps max(|a| + |b|) of its operand pairs, and scales and rounds that maximum once;
+    the global scale must still equal the oracle's bit for bit."""
     rows, K = 16384, 1024
     x = W.with_outliers((rows, K), 0.005, 30.0, W._gen(rows * 3 + group, "cpu"), "cpu")
     check(oracle, x, group, None)
