@@ -60,9 +60,10 @@ METRIC = "nvfp4_linear TFLOPS (% of dense FP4 peak); quantizer GB/s (% of HBM)"
 # only for the kernel sources it was taken on (sha256 prefix); reported as null once a
 # source has changed.
 MEASURED_TRAFFIC = {
-    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "", "bytes_per_step": None},
-    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "",
-              "bytes_per_step": None},
+    "gemm": {"src": "nvfp4_block_scaled_17_b200/csrc/gemm.cu", "sha": "9f24da6eab1ac096",
+             "bytes_per_step": 673.5e6},
+    "quant": {"src": "nvfp4_block_scaled_17_b200/csrc/quantize.cu", "sha": "ac97f3161a1cc410",
+              "bytes_per_step": 812.5e6},
 }
 
 GROUP = 128

@@ -431,7 +431,14 @@ struct RowParams {
     uint32_t n_items;       // ceil(total_units / 32)
     uint32_t upr;           // units per row, K / 128
     FastDiv upr_div;
+    uint32_t reverse;       // 1: visit the items last to first
 };
+
+// The item visited as the j-th of the pass.  The encode pass after an amax pass walks the
+// items in reverse: the amax pass's last items are the ones still in L2.
+__device__ __forceinline__ uint32_t item_at(const RowParams& t, uint32_t j) {
+    return t.reverse ? t.n_items - 1 - j : j;
+}
 
 // fp32 bit pattern of bf16(a) (round to nearest even): a goes to the upper half of the
 // packed pair, +0 to the lower half.
@@ -644,13 +651,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (lane == 0)
         for (int s = 0; s < kRSlots; ++s) {
             const uint32_t it = first + s * stride;
-            if (it < t.n_items) load_item(ring + s * kRItemBytes, &tmE, &tmO, &bars[s], it, policy);
+            if (it < t.n_items)
+                load_item(ring + s * kRItemBytes, &tmE, &tmO, &bars[s], item_at(t, it), policy);
         }
 
     uint32_t tmax = 0u;       // packed bf16 maxima (G = 0)
     float fmax_rot = 0.0f;    // pre-scale rotated maximum (G > 0)
     uint32_t k = 0;
-    for (uint32_t item = first; item < t.n_items; item += stride, ++k) {
+    for (uint32_t j = first; j < t.n_items; j += stride, ++k) {
+        const uint32_t item = item_at(t, j);
         const int s = (int)(k % kRSlots);
         if (!mbar_wait_bounded(&bars[s], (k / kRSlots) & 1u, &s_abort, status, kTmaWaitBudgetNs))
             break;
@@ -659,10 +668,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
         load_unit(slot, lane, w);
         __syncwarp();
         if (lane == 0) {
-            const uint32_t nxt = item + kRSlots * stride;
+            const uint32_t nxt = j + kRSlots * stride;
             if (nxt < t.n_items) {
                 fence_proxy_async_smem();
-                load_item(slot, &tmE, &tmO, &bars[s], nxt, policy);
+                load_item(slot, &tmE, &tmO, &bars[s], item_at(t, nxt), policy);
             }
         }
         // units past the end were zero-filled by the copy: they add nothing to the amax
@@ -999,6 +1008,7 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
         t.n_items = (uint32_t)((n_units + 31) / 32);
         t.upr = (uint32_t)(K / 128);
         t.upr_div = make_fastdiv(t.upr);
+        t.reverse = 0;
         // dynamic scale that fits on chip: one pass, every warp holding at most kRSlots items
         if (gsf_in == nullptr && (int64_t)t.n_items <= (int64_t)dev.sms * kRWarps * kRSlots) {
             // one CTA when its slots hold the whole call (no grid barrier: an ordinary
@@ -1019,6 +1029,7 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
             if (st != NVFP4_OK) return st;
             p.partials = partials;
             p.n_partials = grid;
+            t.reverse = 1;   // the encode pass starts where the amax pass ended (in L2)
         }
         return dispatch_row<1>(group, mE, mO, p, t, grid, dev.device, status, stream);
     }
