@@ -357,15 +357,17 @@ def timed_steps(layers, dynamic, steps, warmup, dist_on):
 
 
 def quantizer_launches(M, K, group, dynamic, sms=148):
-    """Kernel launches one nvfp4_quantize call makes: the encode pass, plus the amax pass
-    for a dynamic scale unless the call fits the single-pass kernel (rows of whole
-    128-value units, 12 warps per SM each holding at most 2 items of 32 units)."""
+    """Kernel launches one nvfp4_quantize call makes: one for a static scale, for a dynamic
+    call that fits the single pass, or for an unrotated dynamic call on rows of whole
+    128-value units (amax and encode phases in one kernel); two (amax pass, encode pass)
+    for other dynamic calls."""
     if not dynamic:
         return 1
-    if K % 128:
-        return 2
-    items = -(-(M * (K // 128)) // 32)
-    return 1 if items <= sms * 12 * 2 else 2
+    if K % 128 == 0:
+        items = -(-(M * (K // 128)) // 32)
+        if items <= sms * 12 * 2 or group == 0:
+            return 1
+    return 2
 
 
 def max_over_ranks(v: float, dist_on: bool) -> float:

@@ -152,7 +152,8 @@ def test_format_conversions_exhaustive(oracle):
 def test_dynamic_single_pass_capacity_edge(oracle, group, rows):
     """A dynamic-scale call that fits on chip takes the single-pass kernel (up to 14.5 M
     values on 148 SMs: 14208 x 1024 is exactly the capacity); 14336 x 1024 is just past it
-    and takes the two passes.  Both bit for bit against the oracle."""
+    and takes the amax phase then the encode phase (one cooperative kernel when unrotated,
+    two launches when rotated).  Both bit for bit against the oracle."""
     K = 1024
     x = W.with_outliers((rows, K), 0.005, 30.0, W._gen(rows + group, "cpu"), "cpu")
     p, sf, g = nv.nvfp4_quantize(x.to(DEV), group, None)
