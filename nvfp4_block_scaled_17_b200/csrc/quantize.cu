@@ -412,8 +412,10 @@ __global__ void __launch_bounds__(kThreads) unit_kernel(const UnitParams p) {
 // further) for the second 64.  An item is 32 consecutive units, one per lane: one 4 KiB
 // box from each map, 128-byte swizzle, so lane t reads row t of each box and the eight
 // lanes of a quarter-warp hit eight distinct 16-byte bank groups.  Every warp keeps its
-// own ring of kRSlots items and issues the load of item k + kRSlots as soon as its lanes
-// have read item k into registers.  One CTA of kRWarps warps per SM, persistent.
+// own ring of kRSlots items and issues the load of its piece r + kRSlots as soon as its
+// lanes have read piece r into registers.  One CTA of kRWarps warps per SM, persistent.
+// These kernels run the single pass of small dynamic calls for every g and the two
+// streaming passes for g = 128; the streaming passes of g <= 64 use the half-unit form.
 // ---------------------------------------------------------------------------
 
 constexpr int kRWarps = 12;
@@ -428,16 +430,17 @@ static_assert(kRSmem <= 232448, "dynamic shared memory above the 227 KiB a CTA c
 
 struct RowParams {
     uint32_t total_units;   // rows * K / 128  (< 2^31)
-    uint32_t n_items;       // ceil(total_units / 32)
+    uint32_t n_items;       // items of the pass (32 units each; 16 in the half-unit form)
     uint32_t upr;           // units per row, K / 128
     FastDiv upr_div;
     uint32_t reverse;       // 1: visit the items last to first
 };
 
-// The item visited as the j-th of the pass.  The encode pass after an amax pass walks the
-// items in reverse: the amax pass's last items are the ones still in L2.
-__device__ __forceinline__ uint32_t item_at(const RowParams& t, uint32_t j) {
-    return t.reverse ? t.n_items - 1 - j : j;
+// The streaming passes hand item j to warp slot j % W (W warps in the grid), and slot q is
+// warp q / gridDim.x of CTA q % gridDim.x: the items of a last, partial round spread over
+// all CTAs first, so every SM gets the same number of items to within one.
+__device__ __forceinline__ uint32_t warp_slot(int warp) {
+    return (uint32_t)warp * gridDim.x + blockIdx.x;
 }
 
 // fp32 bit pattern of bf16(a) (round to nearest even): a goes to the upper half of the
@@ -606,22 +609,27 @@ __device__ __forceinline__ void zero_padding_scales(const UnitParams& p) {
     }
 }
 
+// The 32 units from `base` (rows past the end of x arrive as zeros).
+__device__ __forceinline__ void load_units(uint8_t* slot, const CUtensorMap* tmE,
+                                           const CUtensorMap* tmO, uint64_t* bar, uint32_t base,
+                                           uint64_t policy) {
+    mbar_arrive_expect_tx(bar, kRItemBytes);
+    tma_load_2d_hint(slot, tmE, bar, 0, (int32_t)base, policy);
+    tma_load_2d_hint(slot + kRHalfBytes, tmO, bar, 0, (int32_t)base, policy);
+}
+
 __device__ __forceinline__ void load_item(uint8_t* slot, const CUtensorMap* tmE,
                                           const CUtensorMap* tmO, uint64_t* bar, uint32_t item,
                                           uint64_t policy) {
-    mbar_arrive_expect_tx(bar, kRItemBytes);
-    tma_load_2d_hint(slot, tmE, bar, 0, (int32_t)(item * 32), policy);
-    tma_load_2d_hint(slot + kRHalfBytes, tmO, bar, 0, (int32_t)(item * 32), policy);
+    load_units(slot, tmE, tmO, bar, item * 32, policy);
 }
 
-// MODE 0: amax partials (one per CTA).  MODE 1: quantize.  MODE 4: a dynamic-scale call in
-// one cooperative grid: the amax phase (x loaded with evict_last), the per-CTA maxima at a
-// bounded grid barrier on `arrive` (zeroed before the launch), then the encode phase, which
-// walks the items last to first so that it starts on those still in L2.
+// MODE 0: amax partials (one per CTA).  MODE 1: quantize; after an amax pass it walks the
+// pieces last to first, so that it starts on those still in L2.
 template <int G, int MODE>
 __global__ void __launch_bounds__(kRThreads, 1)
     row_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmO,
-               const UnitParams p, const RowParams t, unsigned int* arrive, int* status) {
+               const UnitParams p, const RowParams t, int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -635,29 +643,36 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (threadIdx.x == 0) s_abort = 0;
     if (lane == 0)
         for (int s = 0; s < kRSlots; ++s) mbar_init(&full[warp * kRSlots + s], 1);
+    if (threadIdx.x == 0) {   // the descriptors do not depend on the previous kernel
+        prefetch_tensormap(&tmE);
+        prefetch_tensormap(&tmO);
+    }
     fence_barrier_init();
     __syncthreads();
     griddep_wait();
     griddep_launch_dependents();
 
     const uint32_t stride = gridDim.x * kRWarps;
+    const uint32_t first = warp_slot(warp);
     uint8_t* ring = smem + warp * kRSlots * kRItemBytes;
     uint64_t* bars = full + warp * kRSlots;
-    const uint32_t first = blockIdx.x * kRWarps + warp;
     uint32_t k = 0;   // uses of this warp's ring so far; slot k % kRSlots, parity (k / kRSlots) & 1
 
-    // One streaming pass over this warp's items (in reverse when asked): the first kRSlots
-    // loads, then per item wait, read into registers, refill the slot, body(item, words).
-    // Returns false after a timeout.
-    auto pass = [&](bool reverse, uint64_t policy, auto&& body) -> bool {
-        auto at = [&](uint32_t j) { return reverse ? t.n_items - 1 - j : j; };
+    // A streaming pass over this warp's items (last to first when `reverse`): prime issues
+    // the first kRSlots loads, run waits for each item, reads it into registers, refills
+    // the slot and calls body(item, words).
+    auto at = [&](bool reverse, uint32_t j) { return reverse ? t.n_items - 1 - j : j; };
+    auto prime = [&](bool reverse, uint64_t policy) {
         if (lane == 0)
-            for (int s = 0; s < kRSlots; ++s) {
+            for (uint32_t s = 0; s < (uint32_t)kRSlots; ++s) {
                 const uint32_t jj = first + s * stride;
                 const int slot = (int)((k + s) % kRSlots);
                 if (jj < t.n_items)
-                    load_item(ring + slot * kRItemBytes, &tmE, &tmO, &bars[slot], at(jj), policy);
+                    load_item(ring + slot * kRItemBytes, &tmE, &tmO, &bars[slot], at(reverse, jj),
+                              policy);
             }
+    };
+    auto run = [&](bool reverse, uint64_t policy, auto&& body) -> bool {
         for (uint32_t j = first; j < t.n_items; j += stride, ++k) {
             const int s = (int)(k % kRSlots);
             if (!mbar_wait_bounded(&bars[s], (k / kRSlots) & 1u, &s_abort, status, kTmaWaitBudgetNs))
@@ -670,10 +685,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 const uint32_t nxt = j + kRSlots * stride;
                 if (nxt < t.n_items) {
                     fence_proxy_async_smem();
-                    load_item(slot, &tmE, &tmO, &bars[s], at(nxt), policy);
+                    load_item(slot, &tmE, &tmO, &bars[s], at(reverse, nxt), policy);
                 }
             }
-            body(at(j), w);
+            body(at(reverse, j), w);
         }
         return true;
     };
@@ -692,17 +707,259 @@ __global__ void __launch_bounds__(kRThreads, 1)
     };
 
     bool ok = true;
+    static_assert(MODE == 0 || MODE == 1, "amax or encode");
+    if constexpr (MODE == 0) {
+        uint32_t tmax = 0u;       // packed bf16 maxima (G = 0)
+        float fmax_rot = 0.0f;    // pre-scale rotated maximum (G > 0)
+        prime(false, l2_policy_evict_last());
+        ok = run(false, l2_policy_evict_last(),
+                 [&](uint32_t item, const uint4 (&w)[16]) { amax_body(item, w, tmax, fmax_rot); });
+        const float mine = G > 0 ? rotated_amax_bf16(fmax_rot, p.hscale) : absmax_of_pair(tmax);
+        const float mx = block_max(mine, red);
+        if (threadIdx.x == 0) p.partials_out[blockIdx.x] = mx;
+    }
+    if constexpr (MODE == 1) {
+        // the prologue's loads go out before the pass's first copies, which would delay them
+        const float gsf = encode_prologue<kRThreads>(p, red, &s_gsf, inv_tab);
+        zero_padding_scales<kRThreads>(p);
+        prime(t.reverse, l2_policy_evict_first());
+        ok = run(t.reverse, l2_policy_evict_first(),
+                 [&](uint32_t item, const uint4 (&w)[16]) { encode_body(item, w, gsf); });
+    }
+    // after a timeout, let this warp's loads still in flight land before the CTA exits
+    if (!ok && lane == 0) {
+        volatile int no_abort = 0;
+        for (uint32_t s = 0; s < (uint32_t)kRSlots; ++s) {
+            const uint32_t kk = k + s;
+            mbar_wait_bounded(&bars[kk % kRSlots], (kk / kRSlots) & 1u, &no_abort, nullptr,
+                              100000000ull);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Half-unit form (K % 128 == 0, multi-pass calls, g <= 64): two threads share a 128-value
+// unit, each owning 64 consecutive values (one 128-byte half).  Every g-group of g <= 64
+// lies inside a half, so the whole butterfly stays in-thread; a thread holds 64 fp32
+// values instead of 128 and a CTA runs kHWarps warps instead of kRWarps.  (For g = 128
+// the h = 64 stage would pair the two halves: swapping 64 fp32 values per thread through
+// shared memory cost more than the extra warps gained, so g = 128 keeps a whole unit per
+// thread.)
+//
+// An item is 16 consecutive units: a [16, 64] box from each half map (128-byte swizzle),
+// 4 KiB.  Lane l owns half l >> 4 of unit l & 15, so the eight lanes of a quarter-warp
+// read eight rows of one box: eight distinct 16-byte bank groups.
+// ---------------------------------------------------------------------------
+
+constexpr int kHWarps = 16;
+constexpr int kHThreads = kHWarps * 32;
+constexpr int kHSlots = 2;
+constexpr int kHBoxBytes = 16 * 128;               // one 64-value half of 16 units
+constexpr int kHItemBytes = 2 * kHBoxBytes;        // 4 KiB: 16 units
+constexpr int kHRingBytes = kHWarps * kHSlots * kHItemBytes;
+constexpr int kHSmem = 1024 + kHRingBytes + kHWarps * kHSlots * 8;
+static_assert(kHSmem <= 232448, "dynamic shared memory above the 227 KiB a CTA can have");
+
+// The 16 units from `base` (rows past the end of x arrive as zeros).
+__device__ __forceinline__ void load_half_units(uint8_t* slot, const CUtensorMap* tmE,
+                                                const CUtensorMap* tmO, uint64_t* bar,
+                                                uint32_t base, uint64_t policy) {
+    mbar_arrive_expect_tx(bar, kHItemBytes);
+    tma_load_2d_hint(slot, tmE, bar, 0, (int32_t)base, policy);
+    tma_load_2d_hint(slot + kHBoxBytes, tmO, bar, 0, (int32_t)base, policy);
+}
+
+// The eight 8-value chunks of this lane's half-unit.
+__device__ __forceinline__ void load_half(const uint8_t* slot, int lane, uint4 (&w)[8]) {
+    const int u = lane & 15;
+    const uint8_t* base = slot + (lane >> 4) * kHBoxBytes + u * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        w[c] = *reinterpret_cast<const uint4*>(base + ((c ^ (u & 7)) << 4));
+}
+
+// Stages h = 1, 2, ... < STOP of the half's butterfly on pairs (2i, 2i + 1).
+template <int STOP>
+__device__ __forceinline__ void half_butterfly(const uint4 (&w)[8], float2 (&v)[32]) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        v[4 * c] = pair_sum_diff(w[c].x);
+        v[4 * c + 1] = pair_sum_diff(w[c].y);
+        v[4 * c + 2] = pair_sum_diff(w[c].z);
+        v[4 * c + 3] = pair_sum_diff(w[c].w);
+    }
+#pragma unroll
+    for (int h = 2; h < STOP; h *= 2)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if ((i & (h / 2)) == 0) bfly2(v[i], v[i + h / 2]);
+}
+
+// Amax of a half-unit.  G = 0: bf16 maxima of the words.  G > 0: the in-thread butterfly
+// up to its last stage, then max(|a| + |b|) over that stage's pairs (see rotate_amax).
+template <int G>
+__device__ __forceinline__ void half_amax(const uint4 (&w)[8], uint32_t& tmax, float& fmax_) {
+    static_assert(G <= 64, "g = 128 groups span both halves of a unit");
+    if constexpr (G == 0) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) tmax = absmax2_bf16(tmax, absmax_word4(w[c]));
+    } else {
+        float2 v[32];
+        half_butterfly<G / 2>(w, v);
+        constexpr int S = G / 4;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if ((i & S) == 0)
+                fmax_ = max3(fmax_, __fadd_rn(fabsf(v[i].x), fabsf(v[i + S].x)),
+                             __fadd_rn(fabsf(v[i].y), fabsf(v[i + S].y)));
+    }
+}
+
+// The half-unit's 64 values as fp32: rotated (every G-group times H / sqrt(G), rounded to
+// bf16) or, for G = 0, the bf16 input itself.
+template <int G>
+__device__ __forceinline__ void half_values(const uint4 (&w)[8], float hscale, float (&r)[64]) {
+    static_assert(G <= 64, "g = 128 groups span both halves of a unit");
+    if constexpr (G == 0) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t q[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                r[8 * c + 2 * k] = bf16lo(q[k]);
+                r[8 * c + 2 * k + 1] = bf16hi(q[k]);
+            }
+        }
+    } else {
+        float2 v[32];
+        half_butterfly<G>(w, v);
+        const float2 hs = make_float2(hscale, hscale);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float2 g = mul2(v[i], hs);
+            r[2 * i] = bf16_round(g.x);
+            r[2 * i + 1] = bf16_round(g.y);
+        }
+    }
+}
+
+// Encode 64 values (bf16-exact) of one half-unit: four 16-value blocks, 32 bytes of codes
+// and the scale word of its 64-value group in the 128x4 layout.
+__device__ __forceinline__ void encode_half64(const float (&r)[64], float gsf,
+                                              const float* inv_tab, const UnitParams& p,
+                                              int64_t row, int64_t e0) {
+    uint32_t s8[4];
+#pragma unroll
+    for (int b = 0; b < 4; b += 2) {
+        const uint32_t s = e4m3_scales2(__fmul_rn(gsf, block_absmax16(r + 16 * b)),
+                                        __fmul_rn(gsf, block_absmax16(r + 16 * b + 16)));
+        s8[b] = s & 0xffu;
+        s8[b + 1] = s >> 8;
+    }
+    uint32_t codes[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const float inv = inv_tab[s8[c >> 1]];   // rn(gsf / dec(s8)); 0 for a zero scale
+        const float2 iv = make_float2(inv, inv);
+        const float* x = r + 8 * c;
+        const float2 a = mul2(make_float2(x[0], x[1]), iv), b = mul2(make_float2(x[2], x[3]), iv);
+        const float2 cc = mul2(make_float2(x[4], x[5]), iv), d = mul2(make_float2(x[6], x[7]), iv);
+        const float q[8] = {a.x, a.y, b.x, b.y, cc.x, cc.y, d.x, d.y};
+        codes[c] = s8[c >> 1] ? e2m1x8_from_f32(q) : 0u;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(p.packed + row * (p.K / 2) + e0 / 2);
+    dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+    const int64_t cg = e0 / 64;
+    const int64_t off = (((row >> 7) * p.cgroups + cg) << 9) + ((row & 31) << 4) +
+                        (((row >> 5) & 3) << 2);
+    *reinterpret_cast<uint32_t*>(p.sf + off) = s8[0] | (s8[1] << 8) | (s8[2] << 16) | (s8[3] << 24);
+}
+
+// MODE 0: amax partials (one per CTA).  MODE 1: quantize.  MODE 4: amax phase, bounded grid
+// barrier on `arrive` (zeroed before the launch; cooperative launch), encode phase.  The
+// RowParams count items of 16 units here.
+template <int G, int MODE>
+__global__ void __launch_bounds__(kHThreads, 1)
+    half_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmO,
+                const UnitParams p, const RowParams t, unsigned int* arrive, int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kHRingBytes);
+    __shared__ float red[32];
+    __shared__ float s_gsf;
+    __shared__ float inv_tab[128];
+    __shared__ int s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) s_abort = 0;
+    if (lane == 0)
+        for (int s = 0; s < kHSlots; ++s) mbar_init(&full[warp * kHSlots + s], 1);
+    if (threadIdx.x == 0) {   // the descriptors do not depend on the previous kernel
+        prefetch_tensormap(&tmE);
+        prefetch_tensormap(&tmO);
+    }
+    fence_barrier_init();
+    __syncthreads();
+    griddep_wait();
+    griddep_launch_dependents();
+
+    const uint32_t stride = gridDim.x * kHWarps;
+    const uint32_t first = warp_slot(warp);
+    uint8_t* ring = smem + warp * kHSlots * kHItemBytes;
+    uint64_t* bars = full + warp * kHSlots;
+    uint32_t k = 0;   // uses of this warp's ring so far; slot k % kHSlots, parity (k / kHSlots) & 1
+
+    // A streaming pass over this warp's items of 16 units (last to first when `reverse`):
+    // prime issues the first kHSlots loads, run waits for each item, reads the lane's
+    // half-unit, refills the slot and calls body(item, words).
+    auto at = [&](bool reverse, uint32_t j) { return reverse ? t.n_items - 1 - j : j; };
+    auto prime = [&](bool reverse, uint64_t policy) {
+        if (lane == 0)
+            for (uint32_t s = 0; s < (uint32_t)kHSlots; ++s) {
+                const uint32_t jj = first + s * stride;
+                const int slot = (int)((k + s) % kHSlots);
+                if (jj < t.n_items)
+                    load_half_units(ring + slot * kHItemBytes, &tmE, &tmO, &bars[slot],
+                                    at(reverse, jj) * 16, policy);
+            }
+    };
+    auto run = [&](bool reverse, uint64_t policy, auto&& body) -> bool {
+        for (uint32_t j = first; j < t.n_items; j += stride, ++k) {
+            const int s = (int)(k % kHSlots);
+            if (!mbar_wait_bounded(&bars[s], (k / kHSlots) & 1u, &s_abort, status, kTmaWaitBudgetNs))
+                return false;
+            uint8_t* slot = ring + s * kHItemBytes;
+            uint4 w[8];
+            load_half(slot, lane, w);
+            __syncwarp();
+            if (lane == 0) {
+                const uint32_t nxt = j + kHSlots * stride;
+                if (nxt < t.n_items) {
+                    fence_proxy_async_smem();
+                    load_half_units(slot, &tmE, &tmO, &bars[s], at(reverse, nxt) * 16, policy);
+                }
+            }
+            body(at(reverse, j), w);
+        }
+        return true;
+    };
+    bool ok = true;
     if constexpr (MODE == 0 || MODE == 4) {
         uint32_t tmax = 0u;       // packed bf16 maxima (G = 0)
         float fmax_rot = 0.0f;    // pre-scale rotated maximum (G > 0)
-        ok = pass(false, l2_policy_evict_last(),
-                  [&](uint32_t item, const uint4 (&w)[16]) { amax_body(item, w, tmax, fmax_rot); });
+        // half-units past the end were zero-filled by the copy: they add nothing
+        prime(false, l2_policy_evict_last());
+        ok = run(false, l2_policy_evict_last(),
+                 [&](uint32_t, const uint4 (&w)[8]) { half_amax<G>(w, tmax, fmax_rot); });
         const float mine = G > 0 ? rotated_amax_bf16(fmax_rot, p.hscale) : absmax_of_pair(tmax);
         const float mx = block_max(mine, red);
         if (threadIdx.x == 0) p.partials_out[blockIdx.x] = mx;
     }
     if constexpr (MODE == 4) {
-        // grid-wide barrier: every CTA publishes its maximum, then waits (bounded) for all
+        // the encode phase's first loads go out before the barrier wait
+        if (ok) prime(true, l2_policy_evict_first());
         if (threadIdx.x == 0) {
             __threadfence();
             atomicAdd(arrive, 1u);
@@ -720,19 +977,30 @@ __global__ void __launch_bounds__(kRThreads, 1)
         if (s_abort) ok = false;
     }
     if constexpr (MODE == 1 || MODE == 4) {
+        const bool rev = MODE == 4 || t.reverse;
         if (ok) {
-            const float gsf = encode_prologue<kRThreads>(p, red, &s_gsf, inv_tab);
-            zero_padding_scales<kRThreads>(p);
-            ok = pass(MODE == 4 || t.reverse, l2_policy_evict_first(),
-                      [&](uint32_t item, const uint4 (&w)[16]) { encode_body(item, w, gsf); });
+            // the prologue's loads go out before the pass's first copies, which would delay
+            // them (MODE 4 issued its first copies before the barrier wait)
+            const float gsf = encode_prologue<kHThreads>(p, red, &s_gsf, inv_tab);
+            zero_padding_scales<kHThreads>(p);
+            if constexpr (MODE == 1) prime(rev, l2_policy_evict_first());
+            ok = run(rev, l2_policy_evict_first(), [&](uint32_t item, const uint4 (&w)[8]) {
+                const uint32_t unit = item * 16 + (lane & 15);
+                if (unit < t.total_units) {
+                    float r[64];
+                    half_values<G>(w, p.hscale, r);
+                    const uint32_t row = fast_div(unit, t.upr_div);
+                    encode_half64(r, gsf, inv_tab, p, (int64_t)row,
+                                  (int64_t)(unit - row * t.upr) * 128 + 64 * (lane >> 4));
+                }
+            });
         }
     }
-    // after a timeout, let this warp's loads still in flight land before the CTA exits
     if (!ok && lane == 0) {
         volatile int no_abort = 0;
-        for (uint32_t s = 0; s < (uint32_t)kRSlots; ++s) {
+        for (uint32_t s = 0; s < (uint32_t)kHSlots; ++s) {
             const uint32_t kk = k + s;
-            mbar_wait_bounded(&bars[kk % kRSlots], (kk / kRSlots) & 1u, &no_abort, nullptr,
+            mbar_wait_bounded(&bars[kk % kHSlots], (kk / kHSlots) & 1u, &no_abort, nullptr,
                               100000000ull);
         }
     }
@@ -932,56 +1200,76 @@ nvfp4_status dispatch_row_single(int g, const CUtensorMap& mE, const CUtensorMap
     return NVFP4_ERR_INVALID_ARG;
 }
 
+template <int G, int MODE>
+nvfp4_status launch_row(const CUtensorMap& mE, const CUtensorMap& mO, const UnitParams& p,
+                        const RowParams& t, int grid, int device, int* status, cudaStream_t stream) {
+    static std::atomic<int> attr_set[64];
+    if (device < 0 || device >= 64) return NVFP4_ERR_DEVICE;
+    if (!set_smem_once(row_kernel<G, MODE>, attr_set, device, kRSmem)) return NVFP4_ERR_CUDA;
+    if (launch_pdl(row_kernel<G, MODE>, (unsigned)grid, kRThreads, kRSmem, stream, mE, mO, p, t,
+                   status) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
+
+// The whole-unit streaming passes serve g = 128 (a group spans a whole unit).
+template <int MODE>
+nvfp4_status dispatch_row(int g, const CUtensorMap& mE, const CUtensorMap& mO, const UnitParams& p,
+                          const RowParams& t, int grid, int device, int* status,
+                          cudaStream_t stream) {
+    if (g == 128) return launch_row<128, MODE>(mE, mO, p, t, grid, device, status, stream);
+    return NVFP4_ERR_INVALID_ARG;
+}
+
 // MODE 4 is a cooperative launch (its CTAs meet at a grid barrier, so all must be resident)
 // after a 4-byte memset of the arrival counter; the others use programmatic dependent
 // launch.
 template <int G, int MODE>
-nvfp4_status launch_row(const CUtensorMap& mE, const CUtensorMap& mO, const UnitParams& p,
-                        const RowParams& t, int grid, int device, unsigned int* arrive, int* status,
-                        cudaStream_t stream) {
+nvfp4_status launch_half(const CUtensorMap& mE, const CUtensorMap& mO, const UnitParams& p,
+                         const RowParams& t, int grid, int device, unsigned int* arrive, int* status,
+                         cudaStream_t stream) {
     static std::atomic<int> attr_set[64];
     if (device < 0 || device >= 64) return NVFP4_ERR_DEVICE;
-    if (!set_smem_once(row_kernel<G, MODE>, attr_set, device, kRSmem)) return NVFP4_ERR_CUDA;
+    if (!set_smem_once(half_kernel<G, MODE>, attr_set, device, kHSmem)) return NVFP4_ERR_CUDA;
     if constexpr (MODE == 4) {
         if (cudaMemsetAsync(arrive, 0, sizeof(unsigned int), stream) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         void* args[] = {const_cast<CUtensorMap*>(&mE), const_cast<CUtensorMap*>(&mO),
                         const_cast<UnitParams*>(&p), const_cast<RowParams*>(&t), &arrive, &status};
-        if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(row_kernel<G, MODE>), dim3(grid),
-                                        dim3(kRThreads), args, kRSmem, stream) != cudaSuccess)
+        if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(half_kernel<G, MODE>), dim3(grid),
+                                        dim3(kHThreads), args, kHSmem, stream) != cudaSuccess)
             return NVFP4_ERR_CUDA;
         return NVFP4_OK;
     }
-    if (launch_pdl(row_kernel<G, MODE>, (unsigned)grid, kRThreads, kRSmem, stream, mE, mO, p, t,
+    if (launch_pdl(half_kernel<G, MODE>, (unsigned)grid, kHThreads, kHSmem, stream, mE, mO, p, t,
                    arrive, status) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
 }
 
 template <int MODE>
-nvfp4_status dispatch_row(int g, const CUtensorMap& mE, const CUtensorMap& mO, const UnitParams& p,
-                          const RowParams& t, int grid, int device, unsigned int* arrive,
-                          int* status, cudaStream_t stream) {
+nvfp4_status dispatch_half(int g, const CUtensorMap& mE, const CUtensorMap& mO, const UnitParams& p,
+                           const RowParams& t, int grid, int device, unsigned int* arrive,
+                           int* status, cudaStream_t stream) {
     switch (g) {
-        case 0: return launch_row<0, MODE>(mE, mO, p, t, grid, device, arrive, status, stream);
-        case 16: return launch_row<16, MODE>(mE, mO, p, t, grid, device, arrive, status, stream);
-        case 32: return launch_row<32, MODE>(mE, mO, p, t, grid, device, arrive, status, stream);
-        case 64: return launch_row<64, MODE>(mE, mO, p, t, grid, device, arrive, status, stream);
-        case 128: return launch_row<128, MODE>(mE, mO, p, t, grid, device, arrive, status, stream);
+        case 0: return launch_half<0, MODE>(mE, mO, p, t, grid, device, arrive, status, stream);
+        case 16: return launch_half<16, MODE>(mE, mO, p, t, grid, device, arrive, status, stream);
+        case 32: return launch_half<32, MODE>(mE, mO, p, t, grid, device, arrive, status, stream);
+        case 64: return launch_half<64, MODE>(mE, mO, p, t, grid, device, arrive, status, stream);
         default: break;
     }
     return NVFP4_ERR_INVALID_ARG;
 }
 
 // One half of every 128-value unit of x: [n_units, 64] bf16 rows 256 bytes apart, based at
-// x (first halves) or x + 128 bytes (second halves), with a [32, 64] box and the 128-byte
-// swizzle.
-bool make_half_map(CUtensorMap* map, const void* base, int64_t n_units) {
+// x (first halves) or x + 128 bytes (second halves), with a [box_rows, 64] box and the
+// 128-byte swizzle.
+bool make_half_map(CUtensorMap* map, const void* base, int64_t n_units, uint32_t box_rows) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {64, (cuuint64_t)n_units};
     cuuint64_t strides[1] = {256};
-    cuuint32_t box[2] = {64, 32};
+    cuuint32_t box[2] = {64, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1047,11 +1335,11 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
         int* status = nullptr;
         if ((st = status_word(&status)) != NVFP4_OK) return st;
         CUtensorMap mE, mO;
-        if (!make_half_map(&mE, x, n_units) ||
-            !make_half_map(&mO, static_cast<const uint8_t*>(x) + 128, n_units))
+        if (!make_half_map(&mE, x, n_units, 32) ||
+            !make_half_map(&mO, static_cast<const uint8_t*>(x) + 128, n_units, 32))
             return NVFP4_ERR_CUDA;
         p.total_units = n_units;
-        RowParams t;
+        RowParams t{};
         t.total_units = (uint32_t)n_units;
         t.n_items = (uint32_t)((n_units + 31) / 32);
         t.upr = (uint32_t)(K / 128);
@@ -1068,32 +1356,46 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
                                        (int)(g1 < dev.sms ? (g1 > 0 ? g1 : 1) : dev.sms), partials,
                                        dev.device, status, stream);
         }
-        const int64_t need = ((int64_t)t.n_items + kRWarps - 1) / kRWarps;
+        // multi-pass calls.  g = 128 keeps a whole unit per thread (row_kernel, pieces of 32
+        // units); g <= 64 has every group inside a 64-value half and runs the half-unit
+        // kernels (half_kernel, pieces of 16 units, 16 warps per SM).
+        const bool whole = group == 128;
+        const uint32_t iu = whole ? 32u : 16u;
+        const int warps = whole ? kRWarps : kHWarps;
+        if (!whole && (!make_half_map(&mE, x, n_units, 16) ||
+                       !make_half_map(&mO, static_cast<const uint8_t*>(x) + 128, n_units, 16)))
+            return NVFP4_ERR_CUDA;
+        t.n_items = (uint32_t)((n_units + iu - 1) / iu);
+        const int64_t need = ((int64_t)t.n_items + warps - 1) / warps;
         const int grid = (int)(need < dev.sms ? (need > 0 ? need : 1) : dev.sms);
-        // the arrival counter lives in the last word of the caller's 4 KiB workspace
-        unsigned int* arrive = reinterpret_cast<unsigned int*>(partials) + (kMaxPartials - 1);
+        // the grid-barrier arrival counter lives in the last word of the caller's 4 KiB
+        // workspace (a static call has none and needs none)
+        unsigned int* arrive =
+            partials ? reinterpret_cast<unsigned int*>(partials) + (kMaxPartials - 1) : nullptr;
         if (gsf_in == nullptr && group == 0) {
             // amax phase, grid barrier, encode phase in one cooperative kernel: for the
             // bandwidth-bound unrotated calls (weight packing) this saves a launch, a ramp-up
-            // and a tail (0.76 -> 0.79 of HBM on a Qwen3-VL layer)
+            // and a tail
             p.partials_out = partials;
             p.partials = partials;
             p.n_partials = grid;
-            return launch_row<0, 4>(mE, mO, p, t, grid, dev.device, arrive, status, stream);
+            return launch_half<0, 4>(mE, mO, p, t, grid, dev.device, arrive, status, stream);
         }
         if (gsf_in == nullptr) {
             // rotated: two launches, the amax pass then the encode pass, both with
             // programmatic dependent launch (a cooperative launch cannot overlap the previous
-            // kernel's tail, which cost the ViT block's 33.5 M-value activations 4 %)
+            // kernel's tail)
             UnitParams a = p;
             a.partials_out = partials;
-            st = dispatch_row<0>(group, mE, mO, a, t, grid, dev.device, arrive, status, stream);
+            st = whole ? dispatch_row<0>(group, mE, mO, a, t, grid, dev.device, status, stream)
+                       : dispatch_half<0>(group, mE, mO, a, t, grid, dev.device, arrive, status, stream);
             if (st != NVFP4_OK) return st;
             p.partials = partials;
             p.n_partials = grid;
             t.reverse = 1;   // the encode pass starts where the amax pass ended (in L2)
         }
-        return dispatch_row<1>(group, mE, mO, p, t, grid, dev.device, arrive, status, stream);
+        return whole ? dispatch_row<1>(group, mE, mO, p, t, grid, dev.device, status, stream)
+                     : dispatch_half<1>(group, mE, mO, p, t, grid, dev.device, arrive, status, stream);
     }
 
     if (gsf_in == nullptr) {
