@@ -368,9 +368,11 @@ static nvfp4_status linear_impl(const void* x, int64_t M, int64_t K, const uint8
     st = launch_quantize(x, M, K, group, gsf_x, &scalars[0], xp, xsf, partials, gsf_w, &scalars[1],
                          s);
     if (st != NVFP4_OK) return st;
+    // the weights were complete before the quantizer began: the GEMM may load them early
     if (prepared)
-        return launch_gemm_prepared(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s);
-    return launch_gemm(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s);
+        return launch_gemm_prepared(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s,
+                                    true);
+    return launch_gemm(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s, true);
 }
 
 nvfp4_status nvfp4_linear(const void* x, int64_t M, int64_t K, const uint8_t* w_packed,
@@ -419,7 +421,7 @@ nvfp4_status nvfp4_linear_fixed_scratch(const void* x, int64_t M, int64_t K,
     st = launch_quantize(x, M, K, group, gsf_x, &scalars[0], xp, xsf, partials, gsf_w, &scalars[1],
                          s);
     if (st != NVFP4_OK) return st;
-    return launch_gemm(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s);
+    return launch_gemm(xp, xsf, w_packed, w_sf, &scalars[1], bias, y, M, N, K, s, true);
 }
 
 nvfp4_status nvfp4_debug_gemm_f32(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,

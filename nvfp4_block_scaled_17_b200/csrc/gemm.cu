@@ -43,7 +43,10 @@
 // full wave persistent and splits the leftover tiles that way right behind it.
 //
 // Launches use programmatic stream serialization: set-up overlaps the previous
-// kernel's tail, and griddepcontrol.wait precedes every global access.
+// kernel's tail, and griddepcontrol.wait precedes every global access -- except, when the
+// caller says the weights were complete before the previous kernel began (the linear
+// paths, whose previous kernel is their own activation quantizer), the first stages' B
+// copies, which go out before the wait and overlap the quantizer.
 //
 // Every wait is bounded (globaltimer); on expiry the kernel records
 // NVFP4_ERR_TIMEOUT, drains its own copies and MMAs, frees tensor memory and exits.
@@ -121,6 +124,9 @@ struct GemmParams {
     // int8 operands (the W8A8 linear): fp32 row scales of A and of B
     const float* sx;
     const float* sw;
+    // 1: the weight operand (B and its scales) was complete before the previous kernel on
+    // the stream started, so the producer loads the first stages' B before waiting for it
+    int w_early;
     int* status;
     uint64_t budget_ns;
 };
@@ -211,8 +217,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    griddep_wait();
-    griddep_launch_dependents();
 
     const int num_tiles = p.tile_count;
     // This CTA's work: whole tiles, persistent over the grid; or (split-K) the K range
@@ -224,46 +228,77 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int kt_begin = SPLITK ? rank * p.k_tiles / splits : 0;
     const int kt_end = SPLITK ? (rank + 1) * p.k_tiles / splits : p.k_tiles;
 
+    // One stage's B copies: the B box and its scales (per 128-row half, or with RSB one
+    // 4 KiB prepared slot per step), completing on full[stage].
+    auto load_b = [&](int stage, int kt, int n_blk, int steps, int sfb_tiles) {
+        tma_load_2d(sB + stage * SMEM_B, &tmB, &full[stage], kt * BKB, n_blk * BN);
+        if constexpr (!I8) {
+            if constexpr (RSB) {
+                bulk_load(sSFB + stage * SM::SFB, p.sfb + ((size_t)n_blk * p.kchunks + 4 * kt) * 4096,
+                          (uint32_t)steps * 4096u, &full[stage]);
+            } else {
+                for (int t = 0; t < sfb_tiles; ++t)
+                    bulk_load(sSFB + stage * SM::SFB + t * 2048,
+                              p.sfb + ((size_t)(2 * n_blk + t) * p.kchunks + 4 * kt) * 512,
+                              (uint32_t)steps * 512u, &full[stage]);
+            }
+        }
+    };
+    auto stage_bytes = [&](int steps, int sfb_tiles) -> uint32_t {
+        const uint32_t sf_bytes = I8 ? 0u : (uint32_t)steps * 512u;
+        const uint32_t sfb_bytes = I8 ? 0u : (RSB ? (uint32_t)steps * 4096u : sf_bytes * sfb_tiles);
+        return SMEM_A + SMEM_B + sf_bytes + sfb_bytes;
+    };
+    // With w_early the producer issues the first tile's first stages of B before waiting
+    // for the previous kernel (which wrote A, not B); their A copies follow the wait.
+    int n_early = 0;
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        if (p.w_early && tile_first < num_tiles) {
+            int m_blk, n_blk;
+            tile_coords(p, p.tile_base + tile_first, m_blk, n_blk);
+            const int sfb_tiles = (2 * n_blk + 1 < p.sf_row_tiles_b) ? 2 : 1;
+            n_early = min(STAGES, kt_end - kt_begin);
+            for (int i = 0; i < n_early; ++i) {
+                const int kt = kt_begin + i;
+                const int steps = min(4, p.kchunks - 4 * kt);
+                mbar_arrive_expect_tx(&full[i], stage_bytes(steps, sfb_tiles));
+                load_b(i, kt, n_blk, steps, sfb_tiles);
+            }
+        }
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+
     if (warp == 0) {
         if (lane == 0) {
-            prefetch_tensormap(&tmA);
-            prefetch_tensormap(&tmB);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, issued_phase = 0;   // per-stage bit masks
             bool ok = true;
+            int fills = 0;   // stages filled so far; the first n_early already hold B
             for (int tile = tile_first; ok && tile < num_tiles; tile += tile_step) {
                 int m_blk, n_blk;
                 tile_coords(p, p.tile_base + tile, m_blk, n_blk);
                 const int sfb_tiles = (2 * n_blk + 1 < p.sf_row_tiles_b) ? 2 : 1;
-                for (int kt = kt_begin; kt < kt_end; ++kt) {
-                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status,
-                                           p.budget_ns)) {
-                        ok = false;
-                        break;
-                    }
+                for (int kt = kt_begin; kt < kt_end; ++kt, ++fills) {
                     const int steps = min(4, p.kchunks - 4 * kt);
                     const uint32_t sf_bytes = I8 ? 0u : (uint32_t)steps * 512u;
-                    // B scales: per 128-row half, or (RSB) one 4 KiB prepared slot per step
-                    const uint32_t sfb_bytes = RSB ? (uint32_t)steps * 4096u : sf_bytes * sfb_tiles;
-                    mbar_arrive_expect_tx(&full[stage], SMEM_A + SMEM_B + sf_bytes + sfb_bytes);
+                    if (fills >= n_early) {
+                        if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status,
+                                               p.budget_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&full[stage], stage_bytes(steps, sfb_tiles));
+                        load_b(stage, kt, n_blk, steps, sfb_tiles);
+                    }
                     tma_load_2d(sA + stage * SMEM_A, &tmA, &full[stage], kt * BKB, m_blk * BM);
-                    tma_load_2d(sB + stage * SMEM_B, &tmB, &full[stage], kt * BKB, n_blk * BN);
-                    if constexpr (!I8) {
+                    if constexpr (!I8)
                         bulk_load(sSFA + stage * SMEM_SFA,
                                   p.sfa + ((size_t)m_blk * p.kchunks + 4 * kt) * 512, sf_bytes,
                                   &full[stage]);
-                        if constexpr (RSB) {
-                            bulk_load(sSFB + stage * SM::SFB,
-                                      p.sfb + ((size_t)n_blk * p.kchunks + 4 * kt) * 4096,
-                                      sfb_bytes, &full[stage]);
-                        } else {
-                            for (int t = 0; t < sfb_tiles; ++t)
-                                bulk_load(sSFB + stage * SM::SFB + t * 2048,
-                                          p.sfb + ((size_t)(2 * n_blk + t) * p.kchunks + 4 * kt) * 512,
-                                          sf_bytes, &full[stage]);
-                        }
-                    }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -731,7 +766,8 @@ template <bool QOUT, bool I8, bool RSB = false, bool F32 = false>
 nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                               const uint8_t* sfb, const float* alpha, const void* bias, void* y,
                               int64_t M, int64_t N, int64_t K, const QuantOut* q,
-                              const float* sx, const float* sw, cudaStream_t stream) {
+                              const float* sx, const float* sw, cudaStream_t stream,
+                              bool weights_ready = false) {
     DeviceInfo dev;
     nvfp4_status st = device_info(&dev);
     if (st != NVFP4_OK) return st;
@@ -741,7 +777,8 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
     // few activation rows: the swapped-operand kernel (gemm_small.cu)
     if constexpr (!QOUT && !I8) {
         if (M <= kSmallMaxRows)
-            return launch_gemm_small(a, sfa, b, sfb, RSB, F32, alpha, bias, y, M, N, K, stream);
+            return launch_gemm_small(a, sfa, b, sfb, RSB, F32, alpha, bias, y, M, N, K, stream,
+                                     weights_ready);
     }
     const int64_t kbytes = I8 ? K : K / 2;   // bytes of one operand row
     CUtensorMap mapA, mapB, mapY;
@@ -790,6 +827,7 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
         p.q_gsf = q->gsf;
         p.q_cgroups = (int)(N / 64);
     }
+    p.w_early = weights_ready ? 1 : 0;
     p.status = status;
     p.budget_ns = 4000000000ull;   // 4 s
 
@@ -876,17 +914,18 @@ nvfp4_status launch_prepare_scales(const uint8_t* sf, int64_t N, int64_t K, uint
 
 nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          const uint8_t* sfb, const float* alpha, const void* bias, void* y,
-                         int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+                         int64_t M, int64_t N, int64_t K, cudaStream_t stream,
+                         bool weights_ready) {
     return launch_gemm_impl<false, false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, nullptr,
-                                          nullptr, nullptr, stream);
+                                          nullptr, nullptr, stream, weights_ready);
 }
 
 nvfp4_status launch_gemm_prepared(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                                   const uint8_t* sfb_prepared, const float* alpha,
                                   const void* bias, void* y, int64_t M, int64_t N, int64_t K,
-                                  cudaStream_t stream) {
+                                  cudaStream_t stream, bool weights_ready) {
     return launch_gemm_impl<false, false, true>(a, sfa, b, sfb_prepared, alpha, bias, y, M, N, K,
-                                                nullptr, nullptr, nullptr, stream);
+                                                nullptr, nullptr, nullptr, stream, weights_ready);
 }
 
 nvfp4_status launch_gemm_f32(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,

@@ -30,6 +30,9 @@
 //     tile over the S partials in rank order (distributed shared memory) and applies
 //     alpha and the bias: deterministic, and the unrounded-output build (F32) stores
 //     the same fp32 value the bf16 build rounds.
+// With weights_ready (the linear paths) the weight copies of the first stages go out
+// before the wait for the previous kernel, so the weight stream overlaps the activation
+// quantizer; the activation's copies follow the wait.
 // Every wait is bounded; on expiry the kernel records NVFP4_ERR_TIMEOUT, drains its
 // copies and MMAs, frees tensor memory and returns.  No load uses cluster multicast.
 #include <atomic>
@@ -73,6 +76,9 @@ struct SmallParams {
     int kchunks;               // K / 64
     int w_row_tiles;           // ceil(N / 128)
     int splits;
+    // 1: the weights (W and its scales) were complete before the previous kernel on the
+    // stream started, so the producer loads them before waiting for it
+    int w_early;
     int* status;
     uint64_t budget_ns;
 };
@@ -116,8 +122,6 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    griddep_wait();
-    griddep_launch_dependents();
 
     const int splits = p.splits;
     const int rank = (int)cluster_rank();
@@ -126,37 +130,64 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
     const int kt_end = (rank + 1) * p.k_tiles / splits;
     const bool two = 2 * tile + 1 < p.w_row_tiles;   // the second 128-row MMA has rows
 
+    // One stage's weight copies (the W box and its scales), completing on full[stage].
+    auto load_w = [&](int stage, int kt, int steps) {
+        uint8_t* sW = smem + stage * XS_STAGE;
+        uint8_t* sSFW = sW + XS_W + XS_X;
+        tma_load_2d(sW, &tmW, &full[stage], kt * XBKB, tile * XW_ROWS);
+        if constexpr (RSB) {
+            for (int j = 0; j < steps; ++j)
+                bulk_load(sSFW + j * 1024, p.sfw + ((size_t)tile * p.kchunks + 4 * kt + j) * 4096,
+                          1024u, &full[stage]);
+        } else {
+            for (int t = 0; t < (two ? 2 : 1); ++t)
+                bulk_load(sSFW + t * 2048, p.sfw + ((size_t)(2 * tile + t) * p.kchunks + 4 * kt) * 512,
+                          (uint32_t)steps * 512u, &full[stage]);
+        }
+    };
+    auto stage_bytes = [&](int steps) -> uint32_t {
+        const uint32_t sfx_bytes = (uint32_t)steps * 512u;
+        const uint32_t sfw_bytes = RSB ? (uint32_t)steps * 1024u : sfx_bytes * (two ? 2u : 1u);
+        return XS_W + (uint32_t)p.mpad * XBKB + sfw_bytes + sfx_bytes;
+    };
+    // With w_early the weight copies of the first stages go out before the wait for the
+    // previous kernel (which wrote the activation, not the weights); the activation's
+    // copies follow the wait.
+    int n_early = 0;
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmW);
+        prefetch_tensormap(&tmX);
+        if (p.w_early) {
+            n_early = min(XSTAGES, kt_end - kt_begin);
+            for (int i = 0; i < n_early; ++i) {
+                const int kt = kt_begin + i;
+                const int steps = min(4, p.kchunks - 4 * kt);
+                mbar_arrive_expect_tx(&full[i], stage_bytes(steps));
+                load_w(i, kt, steps);
+            }
+        }
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+
     if (warp == 0) {
         if (lane == 0) {
-            prefetch_tensormap(&tmW);
-            prefetch_tensormap(&tmX);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, issued_phase = 0;
             for (int kt = kt_begin; kt < kt_end; ++kt) {
-                if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, p.budget_ns))
-                    break;
-                uint8_t* sW = smem + stage * XS_STAGE;
-                uint8_t* sX = sW + XS_W;
-                uint8_t* sSFW = sX + XS_X;
-                uint8_t* sSFX = sSFW + XS_SFW;
                 const int steps = min(4, p.kchunks - 4 * kt);
-                const uint32_t sfx_bytes = (uint32_t)steps * 512u;
-                const uint32_t sfw_bytes = RSB ? (uint32_t)steps * 1024u : sfx_bytes * (two ? 2u : 1u);
-                mbar_arrive_expect_tx(&full[stage], XS_W + (uint32_t)p.mpad * XBKB + sfw_bytes + sfx_bytes);
-                tma_load_2d(sW, &tmW, &full[stage], kt * XBKB, tile * XW_ROWS);
-                tma_load_2d(sX, &tmX, &full[stage], kt * XBKB, 0);
-                if constexpr (RSB) {
-                    for (int j = 0; j < steps; ++j)
-                        bulk_load(sSFW + j * 1024,
-                                  p.sfw + ((size_t)tile * p.kchunks + 4 * kt + j) * 4096, 1024u,
-                                  &full[stage]);
-                } else {
-                    for (int t = 0; t < (two ? 2 : 1); ++t)
-                        bulk_load(sSFW + t * 2048,
-                                  p.sfw + ((size_t)(2 * tile + t) * p.kchunks + 4 * kt) * 512,
-                                  sfx_bytes, &full[stage]);
+                if (kt - kt_begin >= n_early) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status,
+                                           p.budget_ns))
+                        break;
+                    mbar_arrive_expect_tx(&full[stage], stage_bytes(steps));
+                    load_w(stage, kt, steps);
                 }
+                uint8_t* sX = smem + stage * XS_STAGE + XS_W;
+                uint8_t* sSFX = sX + XS_X + XS_SFW;
+                const uint32_t sfx_bytes = (uint32_t)steps * 512u;
+                tma_load_2d(sX, &tmX, &full[stage], kt * XBKB, 0);
                 bulk_load(sSFX, p.sfx + (size_t)(4 * kt) * 512, sfx_bytes, &full[stage]);
                 issued |= 1u << stage;
                 issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -357,7 +388,8 @@ int small_splits(int tiles, int k_tiles, const DeviceInfo& dev) {
 template <bool RSB, bool F32>
 nvfp4_status launch_small_impl(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                                const uint8_t* sfb, const float* alpha, const void* bias, void* y,
-                               int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+                               int64_t M, int64_t N, int64_t K, cudaStream_t stream,
+                               bool weights_ready) {
     DeviceInfo dev;
     nvfp4_status st = device_info(&dev);
     if (st != NVFP4_OK) return st;
@@ -383,6 +415,7 @@ nvfp4_status launch_small_impl(const uint8_t* a, const uint8_t* sfa, const uint8
     p.k_tiles = (int)((K / 2 + XBKB - 1) / XBKB);
     p.kchunks = (int)(K / 64);
     p.w_row_tiles = (int)((N + 127) / 128);
+    p.w_early = weights_ready ? 1 : 0;
     p.status = status;
     p.budget_ns = 4000000000ull;   // 4 s
     const int tiles = (int)((N + XW_ROWS - 1) / XW_ROWS);
@@ -399,13 +432,14 @@ nvfp4_status launch_small_impl(const uint8_t* a, const uint8_t* sfa, const uint8
 nvfp4_status launch_gemm_small(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                                const uint8_t* sfb, bool sfb_prepared, bool f32_out,
                                const float* alpha, const void* bias, void* y, int64_t M,
-                               int64_t N, int64_t K, cudaStream_t stream) {
+                               int64_t N, int64_t K, cudaStream_t stream, bool weights_ready) {
     if (M < 1 || M > XMAX) return NVFP4_ERR_INVALID_ARG;
+    const bool w = weights_ready;
     if (sfb_prepared)
-        return f32_out ? launch_small_impl<true, true>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream)
-                       : launch_small_impl<true, false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream);
-    return f32_out ? launch_small_impl<false, true>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream)
-                   : launch_small_impl<false, false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream);
+        return f32_out ? launch_small_impl<true, true>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream, w)
+                       : launch_small_impl<true, false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream, w);
+    return f32_out ? launch_small_impl<false, true>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream, w)
+                   : launch_small_impl<false, false>(a, sfa, b, sfb, alpha, bias, y, M, N, K, stream, w);
 }
 
 }  // namespace nvfp4

@@ -50,16 +50,22 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
 nvfp4_status launch_rotate(const void* x, void* y, int64_t rows, int64_t K, int group,
                            cudaStream_t stream);
 
+// weights_ready (here and below): b and sfb were complete before the previous kernel on
+// the stream started -- the linear paths, whose previous kernel is their own activation
+// quantizer, which itself waited for all earlier work -- so the kernel may start loading
+// them before it waits for that kernel.  False for a bare GEMM call, whose predecessor may
+// be the kernel that writes the weights.
 nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          const uint8_t* sfb, const float* alpha, const void* bias, void* y,
-                         int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+                         int64_t M, int64_t N, int64_t K, cudaStream_t stream,
+                         bool weights_ready = false);
 
 // The same GEMM with the weight's scales in the prepared order (launch_prepare_scales):
 // one 128x256b tensor-memory copy per K step for both 128-row halves of a B tile.
 nvfp4_status launch_gemm_prepared(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                                   const uint8_t* sfb_prepared, const float* alpha,
                                   const void* bias, void* y, int64_t M, int64_t N, int64_t K,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, bool weights_ready = false);
 size_t prepared_scale_bytes(int64_t N, int64_t K);
 nvfp4_status launch_prepare_scales(const uint8_t* sf, int64_t N, int64_t K, uint8_t* out,
                                    cudaStream_t stream);
@@ -81,7 +87,8 @@ constexpr int64_t kSmallMaxRows = 32;
 nvfp4_status launch_gemm_small(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                                const uint8_t* sfb, bool sfb_prepared, bool f32_out,
                                const float* alpha, const void* bias, void* y, int64_t M,
-                               int64_t N, int64_t K, cudaStream_t stream);
+                               int64_t N, int64_t K, cudaStream_t stream,
+                               bool weights_ready = false);
 
 // 2-D uint8 tensor map [rows, row_bytes] with a [box_rows, 128-byte] box and the
 // 128-byte swizzle (the GEMM operand loads).

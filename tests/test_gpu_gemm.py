@@ -319,3 +319,26 @@ def test_linear_prepared_bit_exact(group, dynamic):
     torch.cuda.synchronize()
     assert nv.last_device_status() == nv.OK
     assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 5120, 5120), (128, 5120, 5120), (512, 8192, 1024)])
+def test_linear_sees_weights_written_just_before(M, N, K):
+    """The linear's GEMM starts loading the weights before it waits for the activation
+    quantizer, which is safe only because the quantizer itself waits for all earlier
+    work.  Overwrite the weight buffers with another weight on the same stream, with no
+    synchronisation, and call the linear right after: the result must be the second
+    weight's, bit for bit (swapped-operand, split-K and persistent GEMM builds)."""
+    x = W.with_outliers((M, K), 0.01, 20.0, W._gen(M + 7, DEV), DEV)
+    w1 = W.normal((N, K), 0.02, W._gen(N + 8, DEV), DEV).to(torch.bfloat16)
+    w2 = W.normal((N, K), 0.05, W._gen(N + 9, DEV), DEV).to(torch.bfloat16)
+    wp2, wsf2, gw2 = nv.pack_weight(w2, 0)
+    ref = nv.nvfp4_linear(x, wp2, wsf2, gw2, N)
+    torch.cuda.synchronize()
+    wp, wsf, gw = nv.pack_weight(w1, 0)
+    y1 = nv.nvfp4_linear(x, wp, wsf, gw, N)
+    nv.nvfp4_quantize(w2, 0, None, out=(wp, wsf, gw))   # the same buffers, no sync
+    y2 = nv.nvfp4_linear(x, wp, wsf, gw, N)
+    torch.cuda.synchronize()
+    assert nv.last_device_status() == nv.OK
+    assert not torch.equal(y1.view(torch.int16), ref.view(torch.int16))
+    assert torch.equal(y2.view(torch.int16), ref.view(torch.int16))
