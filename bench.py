@@ -358,14 +358,14 @@ def timed_steps(layers, dynamic, steps, warmup, dist_on):
 
 def quantizer_launches(M, K, group, dynamic, sms=148):
     """Kernel launches one nvfp4_quantize call makes: one for a static scale, for a dynamic
-    call that fits the single pass, or for an unrotated dynamic call on rows of whole
-    128-value units (amax and encode phases in one kernel); two (amax pass, encode pass)
-    for other dynamic calls."""
+    call of at most 12 items of 32 units (the one-CTA single pass), or for an unrotated
+    dynamic call on rows of whole 128-value units (amax and encode phases in one kernel);
+    two (amax pass, encode pass) for other dynamic calls."""
     if not dynamic:
         return 1
     if K % 128 == 0:
         items = -(-(M * (K // 128)) // 32)
-        if items <= sms * 12 * 2 or group == 0:
+        if items <= 12 or group == 0:
             return 1
     return 2
 

@@ -1007,21 +1007,21 @@ __global__ void __launch_bounds__(kHThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Single pass for a dynamic scale when the whole call fits in shared memory at once
-// (every warp's items fit its kRSlots ring slots: 148 x 12 x 2 items of 4096 values,
-// 14.5 M values on 148 SMs -- a 4096 x 1024 tile is 4.2 M).  Each warp loads its items
-// once, rotates them in place in shared memory while taking the amax, the CTAs meet at a
-// grid barrier (cooperative launch, so all of them are resident; the wait is bounded),
-// and every warp then encodes its items from shared memory with the global scale: one
-// HBM read and one rotation instead of two.  The arithmetic is the two-pass kernels'
-// own, so the results are identical.
+// Single pass for a small dynamic-scale call: one CTA whose warps hold every item of
+// the call at once (at most kRWarps * kRSlots items of 4096 values; calls of up to kRWarps
+// items are routed here, one item per warp).  Each warp loads its items once, rotates them
+// in place in shared memory while taking the amax, the block reduces the maximum, and
+// every warp encodes its items from shared memory with the global scale: one read, one
+// rotation and one launch, with no grid barrier.  The arithmetic is the streaming passes'
+// own, so the results are identical.  (A multi-CTA form with a grid barrier under a
+// cooperative launch measured slower than the two streaming passes at every size it
+// covered, so larger calls take those.)
 // ---------------------------------------------------------------------------
 
 template <int G>
 __global__ void __launch_bounds__(kRThreads, 1)
     row_single_kernel(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmO,
-                      const UnitParams p, const RowParams t, float* partials,
-                      unsigned int* arrive, int* status) {
+                      const UnitParams p, const RowParams t, int* status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -1035,20 +1035,20 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (threadIdx.x == 0) s_abort = 0;
     if (lane == 0)
         for (int s = 0; s < kRSlots; ++s) mbar_init(&full[warp * kRSlots + s], 1);
+    if (threadIdx.x == 0) {   // the descriptors do not depend on the previous kernel
+        prefetch_tensormap(&tmE);
+        prefetch_tensormap(&tmO);
+    }
     fence_barrier_init();
     __syncthreads();
-    // a one-CTA call is launched with programmatic stream serialization (a cooperative
-    // grid is not): wait for the previous kernel before the first global access
     griddep_wait();
     griddep_launch_dependents();
 
-    const uint32_t stride = gridDim.x * kRWarps;
-    const uint32_t first = blockIdx.x * kRWarps + warp;
     uint8_t* ring = smem + warp * kRSlots * kRItemBytes;
     uint64_t* bars = full + warp * kRSlots;
     if (lane == 0)
         for (int s = 0; s < kRSlots; ++s) {
-            const uint32_t it = first + s * stride;
+            const uint32_t it = warp + s * kRWarps;
             if (it < t.n_items)
                 load_item(ring + s * kRItemBytes, &tmE, &tmO, &bars[s], it, l2_policy_evict_first());
         }
@@ -1057,7 +1057,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     uint32_t tmax = 0u;
     bool ok = true;
     for (int s = 0; s < kRSlots; ++s) {
-        const uint32_t item = first + s * stride;
+        const uint32_t item = warp + s * kRWarps;
         if (item >= t.n_items) break;
         if (!mbar_wait_bounded(&bars[s], 0u, &s_abort, status, kTmaWaitBudgetNs)) {
             ok = false;
@@ -1086,45 +1086,17 @@ __global__ void __launch_bounds__(kRThreads, 1)
         // let this warp's other loads land before the CTA can leave
         volatile int no_abort = 0;
         for (int s = 0; s < kRSlots; ++s)
-            if (first + s * stride < t.n_items)
+            if (warp + s * kRWarps < t.n_items)
                 mbar_wait_bounded(&bars[s], 0u, &no_abort, nullptr, 100000000ull);
     }
 
-    // grid-wide amax: per-CTA partials, then a bounded barrier on the arrival count (a
-    // one-CTA grid needs neither)
+    // the call's amax (warp 0 holds it), the global scale, then the encode table
     const float m = block_max(absmax_of_pair(tmax), red);
-    if (gridDim.x == 1) {
-        if (threadIdx.x == 0) s_gsf = m;
-    } else if (threadIdx.x == 0) {
-        partials[blockIdx.x] = m;
-        __threadfence();
-        atomicAdd(arrive, 1u);
-        const uint64_t t0 = globaltimer_ns();
-        while (atomicAdd(arrive, 0u) < gridDim.x) {
-            if (s_abort || globaltimer_ns() - t0 > kTmaWaitBudgetNs) {
-                record_status(status, NVFP4_ERR_TIMEOUT);
-                s_abort = 1;
-                break;
-            }
-        }
-        __threadfence();
-    }
+    if (threadIdx.x == 0) s_gsf = __fdiv_rn(kFp4E4m3Range, fmaxf(m, kAmaxFloor));
     __syncthreads();
     if (s_abort) return;
-
-    // the global scale from every CTA's partial (read past L1), then the encode table
-    float mm = 0.0f;
-    if (gridDim.x == 1) {
-        mm = s_gsf;   // the block's own maximum, published above
-        __syncthreads();
-    } else {
-        for (int i = threadIdx.x; i < (int)gridDim.x; i += kRThreads) mm = fmaxf(mm, __ldcg(partials + i));
-        mm = block_max(mm, red);
-    }
-    if (threadIdx.x == 0) s_gsf = __fdiv_rn(kFp4E4m3Range, fmaxf(mm, kAmaxFloor));
-    __syncthreads();
     const float gsf = s_gsf;
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (threadIdx.x == 0) {
         if (p.gsf_out) *p.gsf_out = gsf;
         if (p.alpha_out) *p.alpha_out = __fdiv_rn(1.0f, __fmul_rn(gsf, *p.gsf_w));
     }
@@ -1137,7 +1109,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
 
     // encode the own items from shared memory
     for (int s = 0; s < kRSlots; ++s) {
-        const uint32_t item = first + s * stride;
+        const uint32_t item = warp + s * kRWarps;
         if (item >= t.n_items) break;
         const uint32_t unit = item * 32 + lane;
         if (unit >= t.total_units) continue;
@@ -1161,40 +1133,25 @@ bool set_smem_once(Kernel* k, std::atomic<int> (&flags)[64], int device, int byt
 
 template <int G>
 nvfp4_status launch_row_single(const CUtensorMap& mE, const CUtensorMap& mO, const UnitParams& p,
-                               const RowParams& t, int grid, float* partials, int device,
-                               int* status, cudaStream_t stream) {
+                               const RowParams& t, int device, int* status, cudaStream_t stream) {
     static std::atomic<int> attr_set[64];
     if (device < 0 || device >= 64) return NVFP4_ERR_DEVICE;
     if (!set_smem_once(row_single_kernel<G>, attr_set, device, kRSmem)) return NVFP4_ERR_CUDA;
-    // the arrival counter lives in the last word of the caller's 4 KiB workspace
-    unsigned int* arrive = reinterpret_cast<unsigned int*>(partials) + (kMaxPartials - 1);
-    if (grid == 1) {
-        // one CTA: no grid barrier, so no counter to clear and no cooperative launch
-        if (launch_pdl(row_single_kernel<G>, 1u, kRThreads, kRSmem, stream, mE, mO, p, t, partials,
-                       arrive, status) != cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        return NVFP4_OK;
-    }
-    if (cudaMemsetAsync(arrive, 0, sizeof(unsigned int), stream) != cudaSuccess)
-        return NVFP4_ERR_CUDA;
-    void* args[] = {const_cast<CUtensorMap*>(&mE), const_cast<CUtensorMap*>(&mO),
-                    const_cast<UnitParams*>(&p), const_cast<RowParams*>(&t), &partials, &arrive,
-                    &status};
-    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(row_single_kernel<G>), dim3(grid),
-                                    dim3(kRThreads), args, kRSmem, stream) != cudaSuccess)
+    if (launch_pdl(row_single_kernel<G>, 1u, kRThreads, kRSmem, stream, mE, mO, p, t, status) !=
+        cudaSuccess)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
 }
 
 nvfp4_status dispatch_row_single(int g, const CUtensorMap& mE, const CUtensorMap& mO,
-                                 const UnitParams& p, const RowParams& t, int grid,
-                                 float* partials, int device, int* status, cudaStream_t stream) {
+                                 const UnitParams& p, const RowParams& t, int device, int* status,
+                                 cudaStream_t stream) {
     switch (g) {
-        case 0: return launch_row_single<0>(mE, mO, p, t, grid, partials, device, status, stream);
-        case 16: return launch_row_single<16>(mE, mO, p, t, grid, partials, device, status, stream);
-        case 32: return launch_row_single<32>(mE, mO, p, t, grid, partials, device, status, stream);
-        case 64: return launch_row_single<64>(mE, mO, p, t, grid, partials, device, status, stream);
-        case 128: return launch_row_single<128>(mE, mO, p, t, grid, partials, device, status, stream);
+        case 0: return launch_row_single<0>(mE, mO, p, t, device, status, stream);
+        case 16: return launch_row_single<16>(mE, mO, p, t, device, status, stream);
+        case 32: return launch_row_single<32>(mE, mO, p, t, device, status, stream);
+        case 64: return launch_row_single<64>(mE, mO, p, t, device, status, stream);
+        case 128: return launch_row_single<128>(mE, mO, p, t, device, status, stream);
         default: break;
     }
     return NVFP4_ERR_INVALID_ARG;
@@ -1345,17 +1302,9 @@ nvfp4_status launch_quantize(const void* x, int64_t rows, int64_t K, int group,
         t.upr = (uint32_t)(K / 128);
         t.upr_div = make_fastdiv(t.upr);
         t.reverse = 0;
-        // dynamic scale that fits on chip: one pass, every warp holding at most kRSlots items
-        if (gsf_in == nullptr && (int64_t)t.n_items <= (int64_t)dev.sms * kRWarps * kRSlots) {
-            // one CTA when its slots hold the whole call (no grid barrier: an ordinary
-            // launch), else as many CTAs as give every warp one item, up to one per SM
-            const int64_t g1 = (int64_t)t.n_items <= kRWarps * kRSlots
-                                   ? 1
-                                   : ((int64_t)t.n_items + kRWarps - 1) / kRWarps;
-            return dispatch_row_single(group, mE, mO, p, t,
-                                       (int)(g1 < dev.sms ? (g1 > 0 ? g1 : 1) : dev.sms), partials,
-                                       dev.device, status, stream);
-        }
+        // a small dynamic call: one CTA holds it all, one item per warp (one launch)
+        if (gsf_in == nullptr && t.n_items <= (uint32_t)kRWarps)
+            return dispatch_row_single(group, mE, mO, p, t, dev.device, status, stream);
         // multi-pass calls.  g = 128 keeps a whole unit per thread (row_kernel, pieces of 32
         // units); g <= 64 has every group inside a 64-value half and runs the half-unit
         // kernels (half_kernel, pieces of 16 units, 16 warps per SM).

@@ -149,11 +149,10 @@ def test_format_conversions_exhaustive(oracle):
 
 @pytest.mark.parametrize("group", [0, 128])
 @pytest.mark.parametrize("rows", [4096, 14208, 14336])
-def test_dynamic_single_pass_capacity_edge(oracle, group, rows):
-    """A dynamic-scale call that fits on chip takes the single-pass kernel (up to 14.5 M
-    values on 148 SMs: 14208 x 1024 is exactly the capacity); 14336 x 1024 is just past it
-    and takes the amax phase then the encode phase (one cooperative kernel when unrotated,
-    two launches when rotated).  Both bit for bit against the oracle."""
+def test_dynamic_streaming_sizes(oracle, group, rows):
+    """Dynamic-scale calls of 4.2-14.7 M values run the streaming passes (g = 0: amax and
+    encode phases in one cooperative kernel; g = 128: the amax pass, then the encode pass
+    walking the items in reverse).  Bit for bit against the oracle."""
     K = 1024
     x = W.with_outliers((rows, K), 0.005, 30.0, W._gen(rows + group, "cpu"), "cpu")
     p, sf, g = nv.nvfp4_quantize(x.to(DEV), group, None)
@@ -165,12 +164,13 @@ def test_dynamic_single_pass_capacity_edge(oracle, group, rows):
     assert np.array_equal(to_np(p), op) and np.array_equal(to_np(sf), osf)
 
 
-@pytest.mark.parametrize("group", [0, 128])
-@pytest.mark.parametrize("rows", [1, 96, 97, 100])
-def test_dynamic_single_pass_one_cta_edge(oracle, group, rows):
-    """A dynamic call of at most 24 items of 32 units (96 x 1024: 768 units) runs the
-    single-pass kernel as one CTA, with no grid barrier; 97 rows need a 25th item and a
-    cooperative grid of CTAs.  Both bit for bit against the oracle."""
+@pytest.mark.parametrize("group", [0, 16, 128])
+@pytest.mark.parametrize("rows", [1, 47, 48, 49, 100])
+def test_dynamic_single_pass_edge(oracle, group, rows):
+    """A dynamic call of at most 12 items of 32 units (48 x 1024: 384 units) runs the
+    one-CTA single pass, one item per warp; 49 rows need a 13th item and take the
+    streaming passes (half-unit kernels for g <= 64).  Both bit for bit against the
+    oracle."""
     K = 1024
     x = W.with_outliers((rows, K), 0.01, 20.0, W._gen(rows * 5 + group, "cpu"), "cpu")
     check(oracle, x, group, None)
@@ -178,8 +178,8 @@ def test_dynamic_single_pass_one_cta_edge(oracle, group, rows):
 
 @pytest.mark.parametrize("group", [16, 32, 64, 128])
 def test_dynamic_two_pass_rotated(oracle, group):
-    """Past the single-pass capacity (16384 x 1024 = 16.8 M values) a dynamic call runs the
-    amax pass, then the encode pass.  The amax pass stops before the last butterfly stage,
+    """A dynamic call of 16384 x 1024 (16.8 M values) runs the amax pass, then the encode
+    pass (half-unit kernels for g <= 64, whole-unit ones for g = 128).  The amax pass stops before the last butterfly stage,
     keeps max(|a| + |b|) of its operand pairs, and scales and rounds that maximum once;
     the global scale must still equal the oracle's bit for bit."""
     rows, K = 16384, 1024
@@ -202,8 +202,8 @@ def test_dynamic_amax_last_stage_branch(oracle, sign, group, R, K):
     x[1, group + group // 2] = sign
     xb = x.to(torch.bfloat16)
     check(oracle, xb, group, None)
-    # the same rows repeated past the single-pass capacity (14.55 M values on 148 SMs):
-    # the two-pass route, amax pass then encode pass
+    # the same rows repeated to 14.7 M values: the streaming route, amax pass then encode
+    # pass, many items per warp
     if K % 128 == 0:
         rows = 14_700_000 // K + 1
         big = xb.repeat(rows // R + 1, 1)[:rows].contiguous()
