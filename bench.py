@@ -875,8 +875,10 @@ def run_ours(args, dist_on, rank, world, local_rank):
     legs = {}
     if not args.kernels_only:
         s_total, s_q, s_g = timed_steps(layers, False, args.steps, args.warmup, dist_on)
-        e2e_ms, h2d, d2h, up_ms, down_ms = e2e_steps(layers, max(3, args.steps // 4),
-                                                     max(3, args.warmup), dist_on)
+        # the same K steps as the kernel timing: the pipeline's fill and drain (the first
+        # upload, the last download) are spread over all of them
+        e2e_ms, h2d, d2h, up_ms, down_ms = e2e_steps(layers, args.steps, max(3, args.warmup),
+                                                     dist_on)
         if world == 1:      # the other workloads: single-GPU runs only
             for name, fn in LEGS.items():
                 legs[name] = fn(dev, pk, l2)
