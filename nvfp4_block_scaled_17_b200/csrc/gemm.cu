@@ -13,7 +13,8 @@
 //               already is the tensor-memory copy order, so no reshuffle is needed);
 //               or, for prepared weight scales (RSB), the B scales as one 16 KiB bulk
 //               copy of four 4 KiB per-step slots.
-//   warp 1      MMA issuer (one lane): per K=64 step, tcgen05.cp of the step's scale
+//   warp 1      MMA issuer (the whole warp runs the loop converged; one elected lane
+//               issues each operation): per K=64 step, tcgen05.cp of the step's scale
 //               chunks into a ring of five tensor-memory slots -- A and the two B
 //               halves as 32x128b.warpx4, or with RSB A as warpx4 and both B halves as
 //               one 128x256b copy of the step's slot (the same 8 columns; two copies
@@ -316,7 +317,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        {   // the whole warp runs the issue loop; one elected lane issues (the _w forms)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -326,18 +327,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 const int b = it & 1;
                 const uint32_t use = (uint32_t)(it >> 1);
                 // buffer b fully drained (tile it-2) and the shared columns drained (tile it-1)
-                if (!mbar_wait_bounded(&acc_free[b], (use & 1) ^ 1, abort_flag, p.status,
-                                       p.budget_ns) ||
-                    !mbar_wait_bounded(ovl_free, (uint32_t)(it & 1) ^ 1, abort_flag, p.status,
-                                       p.budget_ns)) {
+                if (!mbar_wait_bounded_warp(&acc_free[b], (use & 1) ^ 1, abort_flag, p.status,
+                                            p.budget_ns) ||
+                    !mbar_wait_bounded_warp(ovl_free, (uint32_t)(it & 1) ^ 1, abort_flag, p.status,
+                                            p.budget_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t acc = tmem + (b ? TMEM_BUF1 : 0u);
                 for (int kt = kt_begin; kt < kt_end; ++kt) {
-                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status,
-                                           p.budget_ns)) {
+                    if (!mbar_wait_bounded_warp(&full[stage], phase, abort_flag, p.status,
+                                                p.budget_ns)) {
                         ok = false;
                         break;
                     }
@@ -349,38 +350,38 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     const uint32_t sfb0 = smem_u32(sSFB + stage * SM::SFB);
                     for (int kk = 0; kk < steps; ++kk) {
                         if constexpr (I8) {
-                            mma_i8(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
-                                   sdesc_kmajor_sw128(b0 + 32 * kk), IDESC_I8,
-                                   kt > kt_begin || kk > 0);
+                            mma_i8_w(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
+                                     sdesc_kmajor_sw128(b0 + 32 * kk), IDESC_I8,
+                                     kt > kt_begin || kk > 0);
                         } else {
                             const uint32_t sfa_t = tmem + TMEM_SF + 12u * (uint32_t)sf_slot;
                             const uint32_t sfb_t = sfa_t + 4;
-                            tc_copy_sf(sfa_t, sdesc_sf(sfa0 + 512 * kk));
+                            tc_copy_sf_w(sfa_t, sdesc_sf(sfa0 + 512 * kk));
                             if constexpr (RSB) {
                                 // both 128-row halves of the step in one copy: the same
                                 // 8 columns the two warpx4 copies below fill
-                                tc_copy_sf_128x256(sfb_t, sdesc_sf_rep(sfb0 + 4096 * kk));
+                                tc_copy_sf_128x256_w(sfb_t, sdesc_sf_rep(sfb0 + 4096 * kk));
                             } else {
-                                tc_copy_sf(sfb_t, sdesc_sf(sfb0 + 512 * kk));
-                                tc_copy_sf(sfb_t + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
+                                tc_copy_sf_w(sfb_t, sdesc_sf(sfb0 + 512 * kk));
+                                tc_copy_sf_w(sfb_t + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
                             }
-                            mma_nvf4(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
-                                     sdesc_kmajor_sw128(b0 + 32 * kk), IDESC, sfa_t, sfb_t,
-                                     kt > kt_begin || kk > 0);
+                            mma_nvf4_w(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
+                                       sdesc_kmajor_sw128(b0 + 32 * kk), IDESC, sfa_t, sfb_t,
+                                       kt > kt_begin || kk > 0);
                             if (++sf_slot == SF_SLOTS) sf_slot = 0;
                         }
                     }
-                    tc_commit(&empty[stage]);
+                    tc_commit_w(&empty[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
                 if (!ok) break;
-                tc_commit(&acc_full[b]);
+                tc_commit_w(&acc_full[b]);
             }
-            // Wait until every tensor-core operation this thread issued has finished.
-            tc_commit(drain);
+            // Wait until every tensor-core operation the warp issued has finished.
+            tc_commit_w(drain);
             volatile int no_abort = 0;
             mbar_wait_bounded(drain, 0, &no_abort, p.status, p.budget_ns);
         }

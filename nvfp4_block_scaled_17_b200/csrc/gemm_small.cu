@@ -24,7 +24,8 @@
 //     slot, which holds both tiles' 128-byte pieces 256 bytes apart (the copy below
 //     reads them with a 256-byte stride, so no replicated bytes cross HBM);
 //   * warp 1 copies each K step's three scale chunks into a five-slot tensor-memory
-//     ring and issues the two MMAs (kind::mxf4nvf4, block16, M = 128, N = M padded);
+//     ring and issues the two MMAs (kind::mxf4nvf4, block16, M = 128, N = M padded),
+//     the whole warp running the loop converged and one elected lane issuing;
 //   * warps 2..9 move the two fp32 partial accumulators into shared memory (the idle
 //     stage buffers), then, after a cluster barrier, each CTA sums its share of the
 //     tile over the S partials in rank order (distributed shared memory) and applies
@@ -205,13 +206,13 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
                 }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        {   // the whole warp runs the issue loop; one elected lane issues (the _w forms)
             int stage = 0;
             uint32_t phase = 0;
             int slot = 0;
             bool ok = true;
             for (int kt = kt_begin; kt < kt_end; ++kt) {
-                if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, p.budget_ns)) {
+                if (!mbar_wait_bounded_warp(&full[stage], phase, abort_flag, p.status, p.budget_ns)) {
                     ok = false;
                     break;
                 }
@@ -224,30 +225,30 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
                 for (int kk = 0; kk < steps; ++kk) {
                     const uint32_t sf_t = tmem + XTMEM_SF + 12u * (uint32_t)slot;
                     if constexpr (RSB) {
-                        tc_copy_sf(sf_t, sdesc_sf_stride(sfw0 + 1024 * kk, 256));
-                        if (two) tc_copy_sf(sf_t + 4, sdesc_sf_stride(sfw0 + 1024 * kk + 128, 256));
+                        tc_copy_sf_w(sf_t, sdesc_sf_stride(sfw0 + 1024 * kk, 256));
+                        if (two) tc_copy_sf_w(sf_t + 4, sdesc_sf_stride(sfw0 + 1024 * kk + 128, 256));
                     } else {
-                        tc_copy_sf(sf_t, sdesc_sf_stride(sfw0 + 512 * kk, 128));
-                        if (two) tc_copy_sf(sf_t + 4, sdesc_sf_stride(sfw0 + 2048 + 512 * kk, 128));
+                        tc_copy_sf_w(sf_t, sdesc_sf_stride(sfw0 + 512 * kk, 128));
+                        if (two) tc_copy_sf_w(sf_t + 4, sdesc_sf_stride(sfw0 + 2048 + 512 * kk, 128));
                     }
-                    tc_copy_sf(sf_t + 8, sdesc_sf_stride(sfx0 + 512 * kk, 128));
+                    tc_copy_sf_w(sf_t + 8, sdesc_sf_stride(sfx0 + 512 * kk, 128));
                     const uint64_t xdesc = sdesc_kmajor_sw128(x0 + 32 * kk);
                     const uint32_t acc = (kt > kt_begin || kk > 0) ? 1u : 0u;
-                    mma_nvf4(tmem, sdesc_kmajor_sw128(w0 + 32 * kk), xdesc, p.idesc, sf_t,
-                             sf_t + 8, acc);
+                    mma_nvf4_w(tmem, sdesc_kmajor_sw128(w0 + 32 * kk), xdesc, p.idesc, sf_t,
+                               sf_t + 8, acc);
                     if (two)
-                        mma_nvf4(tmem + XTMEM_ACC1, sdesc_kmajor_sw128(w0 + 16384 + 32 * kk), xdesc,
-                                 p.idesc, sf_t + 4, sf_t + 8, acc);
+                        mma_nvf4_w(tmem + XTMEM_ACC1, sdesc_kmajor_sw128(w0 + 16384 + 32 * kk),
+                                   xdesc, p.idesc, sf_t + 4, sf_t + 8, acc);
                     if (++slot == XSF_SLOTS) slot = 0;
                 }
-                tc_commit(&empty[stage]);
+                tc_commit_w(&empty[stage]);
                 if (++stage == XSTAGES) {
                     stage = 0;
                     phase ^= 1;
                 }
             }
-            if (ok) tc_commit(acc_full);
-            tc_commit(drain);
+            if (ok) tc_commit_w(acc_full);
+            tc_commit_w(drain);
             volatile int no_abort = 0;
             mbar_wait_bounded(drain, 0, &no_abort, p.status, p.budget_ns);
         }
