@@ -162,12 +162,11 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a, const uint8_t* sfa, const ui
  * nvfp4_prepare_weight_scales -- a weight's 128x4 block scales rearranged once, offline,
  * for nvfp4_gemm_prepared / nvfp4_linear_prepared (same page and operation as
  * nvfp4_gemm; only the order of the B scale bytes differs).  For each 256-row block nb of
- * W and each K step k of 64 values there is one 4 KiB slot, at (nb * K/64 + k) * 4096;
- * inside it, for row group g = 0..15 and half h = 0, 1, the 128 bytes at g*256 + h*128
- * are bytes (g % 4) * 128 .. +127 of the 512-byte 128x4 chunk of row tile 2*nb + h and
- * step k (zero where that row tile is past N).  That is the shared-memory source of one
- * tcgen05.cp 128x256b per K step for both 128-row halves of a B tile, which fills the
- * same tensor-memory columns as two 32x128b.warpx4 copies of the 128x4 chunks.
+ * W and each K stage s of 256 values there is one 4 KiB block, at (nb * ceil(K/256) + s)
+ * * 4096; inside it, the 512 bytes at h*2048 + j*512 (h = 0, 1; j = 0..3) are the 128x4
+ * chunk of row tile 2*nb + h and K step 4*s + j (zero where that row tile is past N or
+ * that step past K/64).  That is the order in which the GEMM holds a stage's B scales in
+ * shared memory, so a stage takes one 4 KiB bulk copy instead of two.
  *   sf  : in,  the weight's 128x4 scales (nvfp4_scale_bytes(N, K) bytes)
  *   out : out, nvfp4_prepared_scale_bytes(N, K) bytes, caller-owned
  *   K % 64 == 0.  Errors: INVALID_ARG, SHAPE, ALIGN (16-byte), DEVICE, CUDA.

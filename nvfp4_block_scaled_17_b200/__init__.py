@@ -208,7 +208,7 @@ def nvfp4_prepared_scale_bytes(N: int, K: int) -> int:
 def prepare_weight_scales(sf: torch.Tensor, N: int, K: int, out: torch.Tensor | None = None,
                           stream=None) -> torch.Tensor:
     """A weight's 128x4 scales in the order nvfp4_gemm_prepared / nvfp4_linear_prepared
-    read (one 4 KiB slot per 256-row block and K step)."""
+    read (one 4 KiB block per 256-row block and 256-value K stage)."""
     if out is None:
         out = torch.empty(max(nvfp4_prepared_scale_bytes(N, K), 1), dtype=torch.uint8,
                           device=sf.device)

@@ -402,10 +402,34 @@ __device__ __forceinline__ void tc_copy_sf_w(uint32_t taddr, uint64_t sdesc) {
                  "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr), "l"(sdesc)
                  : "memory");
 }
-__device__ __forceinline__ void tc_copy_sf_128x256_w(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-                 "@e tcgen05.cp.cta_group::1.128x256b [%0], %1;\n\t}" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
+
+// One K step of the block-scaled MMA, warp-issued with a single election: the step's
+// three scale chunks into tensor memory with 32x128b.warpx4 copies -- A at sfa_t, B's
+// two 128-row halves at sfb_t = sfa_t + 4 and sfa_t + 8, the second half's source
+// descriptor HALF units (16 bytes each) after the first -- then the MMA that reads them.
+template <int HALF>
+__device__ __forceinline__ void mma_step_nvf4_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t sfa_t, uint64_t sfa_desc,
+                                                uint64_t sfb_desc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t"
+        ".reg .pred p, e;\n\t"
+        ".reg .b32 t, u;\n\t"
+        ".reg .b64 s;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "add.u32 t, %5, 4;\n\t"
+        "add.u32 u, %5, 8;\n\t"
+        "add.u64 s, %7, %8;\n\t"
+        "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%5], %6;\n\t"
+        "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [t], %7;\n\t"
+        "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [u], s;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
+        "[t], p;\n\t"
+        "}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_t), "l"(sfa_desc),
+        "l"(sfb_desc), "n"(HALF)
+        : "memory");
 }
 
 // Bounded wait taken by a whole warp: every lane polls, lane 0's outcome decides for all,
@@ -488,21 +512,6 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
 __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t smem_addr) {
     return (uint64_t)((smem_addr >> 4) & 0x3fffu) | ((uint64_t)(1024 >> 4) << 32) |
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// 128 lanes x 256 bits (8 columns) from shared memory, lane l from source row l.
-__device__ __forceinline__ void tc_copy_sf_128x256(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
-}
-
-// Descriptor for tcgen05.cp of a 128-row x 32-byte block stored as 8-row x 16-byte core
-// matrices, core matrix (g, h) (row group g, 16-byte half h) at g * 256 + h * 128: no
-// swizzle, leading-dimension offset 128, stride offset 256.  Read either way round the
-// two offsets stay inside the 4 KiB block.
-__device__ __forceinline__ uint64_t sdesc_sf_rep(uint32_t smem_addr) {
-    return (uint64_t)((smem_addr >> 4) & 0x3fffu) | ((uint64_t)(128 >> 4) << 16) |
-           ((uint64_t)(256 >> 4) << 32) | ((uint64_t)1 << 46);
 }
 
 // Descriptor for tcgen05.cp of a 32-row x 16-byte block: no swizzle, 8-row core

@@ -11,23 +11,24 @@
 //               256 x 128-byte B box (128-byte swizzle), plus the matching 512-byte
 //               chunks of the 128x4 scale layout with plain bulk copies (the layout
 //               already is the tensor-memory copy order, so no reshuffle is needed);
-//               or, for prepared weight scales (RSB), the B scales as one 16 KiB bulk
-//               copy of four 4 KiB per-step slots.
+//               or, for prepared weight scales (RSB), the B scales of the stage as one
+//               4 KiB bulk copy of its prepared block.
 //   warp 1      MMA issuer (the whole warp runs the loop converged; one elected lane
-//               issues each operation): per K=64 step, tcgen05.cp of the step's scale
-//               chunks into a ring of five tensor-memory slots -- A and the two B
-//               halves as 32x128b.warpx4, or with RSB A as warpx4 and both B halves as
-//               one 128x256b copy of the step's slot (the same 8 columns; two copies
-//               per step instead of three) -- then tcgen05.mma
-//               kind::mxf4nvf4 block16 (M=128, N=256, K=64), accumulating in tensor
-//               memory; tcgen05.commit releases the stage and, at the end of a tile,
-//               hands the accumulator to the epilogue.  The copy for step g overwrites
-//               the slot of step g-5, long finished, so the in-order tensor pipe never
-//               waits for an MMA to stop reading the scales it is about to replace.
+//               issues each K step's operations, under a single election): per K=64
+//               step, tcgen05.cp of the step's three scale chunks (A and the two B
+//               halves, 32x128b.warpx4 each) into a ring of five tensor-memory slots,
+//               then tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64),
+//               accumulating in tensor memory; tcgen05.commit releases the stage and,
+//               at the end of a tile, hands the accumulator to the epilogue.  The copy
+//               for step g overwrites the slot of step g-5, long finished, so the
+//               in-order tensor pipe never waits for an MMA to stop reading the scales
+//               it is about to replace.  The issue loop is kept short -- descriptors
+//               advanced by adds, one election per step -- because the single issuing
+//               warp's instruction stream sets the pace at which MMAs reach the pipe.
 //   warps 2..9  epilogue, two warps per 32-lane tensor-memory quadrant (one per
 //               128-column half): tcgen05.ld, alpha, bias, bf16, a 64-byte-swizzled
-//               shared staging tile (two per warp, one with RSB), TMA store (bounds
-//               clipped by the tensor map).
+//               shared staging tile (two per warp), TMA store (bounds clipped by the
+//               tensor map).
 //
 // Accumulator double buffering within 512 tensor-memory columns: tile buffers
 // occupy columns [0, 256) and [192, 448), the scale-factor ring [448, 508).  The two
@@ -74,14 +75,13 @@ constexpr int SMEM_B = BN * BKB;        // 32 KiB
 constexpr int SMEM_SFA = 4 * 512;       // four K=64 scale chunks for 128 rows
 constexpr int STG_BYTES = 32 * 64;      // one 32 x 32 bf16 staging tile
 constexpr int SMEM_BIAS = EPI_WARPS * 256;   // each epilogue warp's 128 bias values of a tile
-// Shared memory of one build.  B scales per stage: four 512-byte chunks per 128-row half
-// in the 128x4 layout; or (RSB, prepared weight scales) one 4 KiB slot per K step, both
-// halves replicated for a single 128x256b copy, which leaves room for one staging tile
-// per epilogue warp instead of two.
+// Shared memory of one build.  B scales per stage: four 512-byte chunks per 128-row half,
+// copied from the 128x4 layout (two bulk copies) or, with RSB (prepared weight scales),
+// as the stage's one 4 KiB block, already in this order.
 template <bool RSB>
 struct GemmSmem {
-    static constexpr int SFB = RSB ? 4 * 4096 : 8 * 512;
-    static constexpr int STG_BUFS = RSB ? 1 : 2;
+    static constexpr int SFB = 4 * 1024;
+    static constexpr int STG_BUFS = 2;
     static constexpr int STG = EPI_WARPS * STG_BUFS * STG_BYTES;
     static constexpr int BYTES =
         1024 + STAGES * (SMEM_A + SMEM_B + SMEM_SFA + SFB) + STG + SMEM_BIAS + 256;
@@ -229,14 +229,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int kt_begin = SPLITK ? rank * p.k_tiles / splits : 0;
     const int kt_end = SPLITK ? (rank + 1) * p.k_tiles / splits : p.k_tiles;
 
-    // One stage's B copies: the B box and its scales (per 128-row half, or with RSB one
-    // 4 KiB prepared slot per step), completing on full[stage].
+    // One stage's B copies: the B box and its scales (per 128-row half, or with RSB the
+    // stage's prepared 4 KiB block), completing on full[stage].
     auto load_b = [&](int stage, int kt, int n_blk, int steps, int sfb_tiles) {
         tma_load_2d(sB + stage * SMEM_B, &tmB, &full[stage], kt * BKB, n_blk * BN);
         if constexpr (!I8) {
             if constexpr (RSB) {
-                bulk_load(sSFB + stage * SM::SFB, p.sfb + ((size_t)n_blk * p.kchunks + 4 * kt) * 4096,
-                          (uint32_t)steps * 4096u, &full[stage]);
+                bulk_load(sSFB + stage * SM::SFB, p.sfb + ((size_t)n_blk * p.k_tiles + kt) * 4096,
+                          4096u, &full[stage]);
             } else {
                 for (int t = 0; t < sfb_tiles; ++t)
                     bulk_load(sSFB + stage * SM::SFB + t * 2048,
@@ -247,7 +247,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     };
     auto stage_bytes = [&](int steps, int sfb_tiles) -> uint32_t {
         const uint32_t sf_bytes = I8 ? 0u : (uint32_t)steps * 512u;
-        const uint32_t sfb_bytes = I8 ? 0u : (RSB ? (uint32_t)steps * 4096u : sf_bytes * sfb_tiles);
+        const uint32_t sfb_bytes = I8 ? 0u : (RSB ? 4096u : sf_bytes * sfb_tiles);
         return SMEM_A + SMEM_B + sf_bytes + sfb_bytes;
     };
     // With w_early the producer issues the first tile's first stages of B before waiting
@@ -344,31 +344,26 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     }
                     tc_fence_after();
                     const int steps = min(4, p.kchunks - 4 * kt);
-                    const uint32_t a0 = smem_u32(sA + stage * SMEM_A);
-                    const uint32_t b0 = smem_u32(sB + stage * SMEM_B);
-                    const uint32_t sfa0 = smem_u32(sSFA + stage * SMEM_SFA);
-                    const uint32_t sfb0 = smem_u32(sSFB + stage * SM::SFB);
-                    for (int kk = 0; kk < steps; ++kk) {
-                        if constexpr (I8) {
-                            mma_i8_w(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
-                                     sdesc_kmajor_sw128(b0 + 32 * kk), IDESC_I8,
-                                     kt > kt_begin || kk > 0);
-                        } else {
-                            const uint32_t sfa_t = tmem + TMEM_SF + 12u * (uint32_t)sf_slot;
-                            const uint32_t sfb_t = sfa_t + 4;
-                            tc_copy_sf_w(sfa_t, sdesc_sf(sfa0 + 512 * kk));
-                            if constexpr (RSB) {
-                                // both 128-row halves of the step in one copy: the same
-                                // 8 columns the two warpx4 copies below fill
-                                tc_copy_sf_128x256_w(sfb_t, sdesc_sf_rep(sfb0 + 4096 * kk));
+                    // Descriptors of the stage's first K step; step kk adds 32 bytes to the
+                    // A and B start addresses and 512 to the scale chunks' (2 and 32 in the
+                    // descriptors' address fields).  B's second 128-row half is 2048 bytes
+                    // (128 units) after the first.
+                    const uint64_t ad = sdesc_kmajor_sw128(smem_u32(sA + stage * SMEM_A));
+                    const uint64_t bd = sdesc_kmajor_sw128(smem_u32(sB + stage * SMEM_B));
+                    const uint64_t sad = sdesc_sf(smem_u32(sSFA + stage * SMEM_SFA));
+                    const uint64_t sbd = sdesc_sf(smem_u32(sSFB + stage * SM::SFB));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        if (kk < steps) {
+                            const uint32_t accumulate = (kt > kt_begin || kk > 0) ? 1u : 0u;
+                            if constexpr (I8) {
+                                mma_i8_w(acc, ad + 2 * kk, bd + 2 * kk, IDESC_I8, accumulate);
                             } else {
-                                tc_copy_sf_w(sfb_t, sdesc_sf(sfb0 + 512 * kk));
-                                tc_copy_sf_w(sfb_t + 4, sdesc_sf(sfb0 + 2048 + 512 * kk));
+                                mma_step_nvf4_w<128>(acc, ad + 2 * kk, bd + 2 * kk, IDESC,
+                                                     tmem + TMEM_SF + 12u * (uint32_t)sf_slot,
+                                                     sad + 32 * kk, sbd + 32 * kk, accumulate);
+                                sf_slot = sf_slot == SF_SLOTS - 1 ? 0 : sf_slot + 1;
                             }
-                            mma_nvf4_w(acc, sdesc_kmajor_sw128(a0 + 32 * kk),
-                                       sdesc_kmajor_sw128(b0 + 32 * kk), IDESC, sfa_t, sfb_t,
-                                       kt > kt_begin || kk > 0);
-                            if (++sf_slot == SF_SLOTS) sf_slot = 0;
                         }
                     }
                     tc_commit_w(&empty[stage]);
@@ -869,33 +864,32 @@ nvfp4_status launch_gemm_impl(const uint8_t* a, const uint8_t* sfa, const uint8_
     return NVFP4_OK;
 }
 
-// Prepared weight scales: the 4 KiB slot of (256-row block nb, K step k) holds, for each
-// 8-row group g (16) and 128-row half h (2), at g * 256 + h * 128, the 128 bytes
-// (g % 4) * 128 .. of the 512-byte 128x4 chunk (row tile 2 nb + h, step k); halves past
-// the last row tile are zero.  One thread per 16 bytes.
+// Prepared weight scales: the 4 KiB block of (256-row block nb, K stage s of 256 values)
+// holds at h * 2048 + j * 512 the 512-byte 128x4 chunk of row tile 2 nb + h and K step
+// 4 s + j -- the order in which a stage's B scales sit in shared memory -- with zeros for
+// row tiles past the last one and steps past K / 64.  One thread per 16 bytes.
 __global__ void __launch_bounds__(256) prepare_scales_kernel(const uint8_t* __restrict__ sf,
                                                              uint8_t* __restrict__ out,
                                                              int64_t pieces, int kchunks,
-                                                             int row_tiles) {
+                                                             int kstages, int row_tiles) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < pieces;
          i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t slot = i >> 8;
+        const int64_t blk = i >> 8;
         const int q = (int)(i & 255);
-        const int g = q >> 4, h = (q >> 3) & 1, part = q & 7;
-        const int64_t nb = slot / kchunks, k = slot - nb * kchunks;
-        const int64_t tile = 2 * nb + h;
+        const int h = q >> 7, j = (q >> 5) & 3, part = q & 31;
+        const int64_t nb = blk / kstages, st = blk - nb * kstages;
+        const int64_t tile = 2 * nb + h, k = 4 * st + j;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (tile < row_tiles)
-            v = *reinterpret_cast<const uint4*>(sf + (tile * kchunks + k) * 512 + (g & 3) * 128 +
-                                                part * 16);
-        *reinterpret_cast<uint4*>(out + slot * 4096 + g * 256 + h * 128 + part * 16) = v;
+        if (tile < row_tiles && k < kchunks)
+            v = *reinterpret_cast<const uint4*>(sf + (tile * kchunks + k) * 512 + part * 16);
+        *reinterpret_cast<uint4*>(out + blk * 4096 + h * 2048 + j * 512 + part * 16) = v;
     }
 }
 
 }  // namespace
 
 size_t prepared_scale_bytes(int64_t N, int64_t K) {
-    return (size_t)((N + 255) / 256) * (size_t)(K / 64) * 4096u;
+    return (size_t)((N + 255) / 256) * (size_t)((K / 64 + 3) / 4) * 4096u;
 }
 
 nvfp4_status launch_prepare_scales(const uint8_t* sf, int64_t N, int64_t K, uint8_t* out,
@@ -904,11 +898,12 @@ nvfp4_status launch_prepare_scales(const uint8_t* sf, int64_t N, int64_t K, uint
     nvfp4_status st = device_info(&dev);
     if (st != NVFP4_OK) return st;
     const int kchunks = (int)(K / 64);
-    const int64_t pieces = (int64_t)((N + 255) / 256) * kchunks * 256;
+    const int kstages = (kchunks + 3) / 4;
+    const int64_t pieces = (int64_t)((N + 255) / 256) * kstages * 256;
     const int64_t need = (pieces + 255) / 256;
     const int64_t cap = (int64_t)dev.sms * 8;
     const int grid = (int)(need < cap ? (need > 0 ? need : 1) : cap);
-    prepare_scales_kernel<<<grid, 256, 0, stream>>>(sf, out, pieces, kchunks,
+    prepare_scales_kernel<<<grid, 256, 0, stream>>>(sf, out, pieces, kchunks, kstages,
                                                     (int)((N + 127) / 128));
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

@@ -20,9 +20,8 @@
 //   * warp 0 loads, per 256-value K stage, the 256 x 128-byte weight box and the
 //     M x 128-byte activation box (128-byte swizzle, rows past M zero-filled), the
 //     activation's 128x4 scale chunks and the weight's: the 128x4 chunks of both row
-//     tiles, or, from prepared weight scales, the first 1 KiB of each step's 4 KiB
-//     slot, which holds both tiles' 128-byte pieces 256 bytes apart (the copy below
-//     reads them with a 256-byte stride, so no replicated bytes cross HBM);
+//     tiles, or, from prepared weight scales, the stage's 4 KiB block (the same chunks
+//     in the same shared-memory order, one bulk copy);
 //   * warp 1 copies each K step's three scale chunks into a five-slot tensor-memory
 //     ring and issues the two MMAs (kind::mxf4nvf4, block16, M = 128, N = M padded),
 //     the whole warp running the loop converged and one elected lane issuing;
@@ -52,7 +51,7 @@ constexpr int XMAX = 128;                    // activation rows at most (the MMA
 constexpr int XTHREADS = 320;
 constexpr int XS_W = XW_ROWS * XBKB;         // 32 KiB
 constexpr int XS_X = XMAX * XBKB;            // 16 KiB
-constexpr int XS_SFW = 4096;                 // two row tiles x four steps x 512 B (or 4 x 1 KiB)
+constexpr int XS_SFW = 4096;                 // two row tiles x four steps x 512 B
 constexpr int XS_SFX = 2048;                 // four steps x 512 B
 constexpr int XS_STAGE = XS_W + XS_X + XS_SFW + XS_SFX;
 constexpr int XSMEM = 1024 + XSTAGES * XS_STAGE + 256;
@@ -83,13 +82,6 @@ struct SmallParams {
     int* status;
     uint64_t budget_ns;
 };
-
-// tcgen05.cp source of a 32-row x 16-byte block whose 8-row core matrices are `stride`
-// bytes apart (128 for a contiguous 128x4 chunk, 256 for a piece of a prepared slot).
-__device__ __forceinline__ uint64_t sdesc_sf_stride(uint32_t smem_addr, uint32_t stride) {
-    return (uint64_t)((smem_addr >> 4) & 0x3fffu) | ((uint64_t)(stride >> 4) << 32) |
-           ((uint64_t)1 << 46);
-}
 
 template <bool RSB, bool F32>
 __global__ void __launch_bounds__(XTHREADS, 1)
@@ -137,9 +129,7 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
         uint8_t* sSFW = sW + XS_W + XS_X;
         tma_load_2d(sW, &tmW, &full[stage], kt * XBKB, tile * XW_ROWS);
         if constexpr (RSB) {
-            for (int j = 0; j < steps; ++j)
-                bulk_load(sSFW + j * 1024, p.sfw + ((size_t)tile * p.kchunks + 4 * kt + j) * 4096,
-                          1024u, &full[stage]);
+            bulk_load(sSFW, p.sfw + ((size_t)tile * p.k_tiles + kt) * 4096, 4096u, &full[stage]);
         } else {
             for (int t = 0; t < (two ? 2 : 1); ++t)
                 bulk_load(sSFW + t * 2048, p.sfw + ((size_t)(2 * tile + t) * p.kchunks + 4 * kt) * 512,
@@ -148,7 +138,7 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
     };
     auto stage_bytes = [&](int steps) -> uint32_t {
         const uint32_t sfx_bytes = (uint32_t)steps * 512u;
-        const uint32_t sfw_bytes = RSB ? (uint32_t)steps * 1024u : sfx_bytes * (two ? 2u : 1u);
+        const uint32_t sfw_bytes = RSB ? 4096u : sfx_bytes * (two ? 2u : 1u);
         return XS_W + (uint32_t)p.mpad * XBKB + sfw_bytes + sfx_bytes;
     };
     // With w_early the weight copies of the first stages go out before the wait for the
@@ -224,14 +214,10 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
                 const uint32_t sfx0 = sfw0 + XS_SFW;
                 for (int kk = 0; kk < steps; ++kk) {
                     const uint32_t sf_t = tmem + XTMEM_SF + 12u * (uint32_t)slot;
-                    if constexpr (RSB) {
-                        tc_copy_sf_w(sf_t, sdesc_sf_stride(sfw0 + 1024 * kk, 256));
-                        if (two) tc_copy_sf_w(sf_t + 4, sdesc_sf_stride(sfw0 + 1024 * kk + 128, 256));
-                    } else {
-                        tc_copy_sf_w(sf_t, sdesc_sf_stride(sfw0 + 512 * kk, 128));
-                        if (two) tc_copy_sf_w(sf_t + 4, sdesc_sf_stride(sfw0 + 2048 + 512 * kk, 128));
-                    }
-                    tc_copy_sf_w(sf_t + 8, sdesc_sf_stride(sfx0 + 512 * kk, 128));
+                    // both weight scale layouts leave the stage's chunks in the same order
+                    tc_copy_sf_w(sf_t, sdesc_sf(sfw0 + 512 * kk));
+                    if (two) tc_copy_sf_w(sf_t + 4, sdesc_sf(sfw0 + 2048 + 512 * kk));
+                    tc_copy_sf_w(sf_t + 8, sdesc_sf(sfx0 + 512 * kk));
                     const uint64_t xdesc = sdesc_kmajor_sw128(x0 + 32 * kk);
                     const uint32_t acc = (kt > kt_begin || kk > 0) ? 1u : 0u;
                     mma_nvf4_w(tmem, sdesc_kmajor_sw128(w0 + 32 * kk), xdesc, p.idesc, sf_t,

@@ -61,7 +61,7 @@ nvfp4_status launch_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                          bool weights_ready = false);
 
 // The same GEMM with the weight's scales in the prepared order (launch_prepare_scales):
-// one 128x256b tensor-memory copy per K step for both 128-row halves of a B tile.
+// one 4 KiB block per 256-row block and 256-value K stage, in shared-memory order.
 nvfp4_status launch_gemm_prepared(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
                                   const uint8_t* sfb_prepared, const float* alpha,
                                   const void* bias, void* y, int64_t M, int64_t N, int64_t K,

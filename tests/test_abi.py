@@ -54,9 +54,9 @@ def test_sizes_match_oracle(L, oracle):
     ws = L.nvfp4_linear_workspace_bytes(4096, 5120)
     assert ws >= 4096 * 5120 // 2 + oracle.scale_bytes(4096, 5120) + 8
     assert ws % 256 == 0
-    # prepared weight scales: one 4 KiB slot per 256-row block and 64-value K step
-    assert L.nvfp4_prepared_scale_bytes(5120, 5120) == 20 * 80 * 4096
-    assert L.nvfp4_prepared_scale_bytes(300, 576) == 2 * 9 * 4096
+    # prepared weight scales: one 4 KiB block per 256-row block and 256-value K stage
+    assert L.nvfp4_prepared_scale_bytes(5120, 5120) == 20 * 20 * 4096
+    assert L.nvfp4_prepared_scale_bytes(300, 576) == 2 * 3 * 4096
     assert L.nvfp4_prepared_scale_bytes(0, 64) == 0 and L.nvfp4_prepared_scale_bytes(8, 48) == 0
 
 

@@ -227,15 +227,19 @@ def test_probe_error_on_gpu():
 
 def prepared_layout_np(sf: np.ndarray, N: int, K: int) -> np.ndarray:
     """The prepared order written out from its definition in the header: per 256-row
-    block nb and K step k a 4 KiB slot; bytes g*256 + h*128 .. +127 of it are bytes
-    (g % 4)*128 .. +127 of the 128x4 chunk (row tile 2 nb + h, step k), zero past N."""
+    block nb and K stage s of 256 values a 4 KiB block; bytes h*2048 + j*512 .. +511 of
+    it are the 128x4 chunk (row tile 2 nb + h, step 4 s + j), zero past N or K/64."""
     kc, tiles, nb = K // 64, (N + 127) // 128, (N + 255) // 256
-    chunks = sf.reshape(-1)[: tiles * kc * 512].reshape(tiles, kc, 4, 128)   # [tile, k, g%4, 128]
-    out = np.zeros((nb, kc, 16, 2, 128), dtype=np.uint8)
-    for h in range(2):
-        t = np.arange(nb) * 2 + h
-        ok = t < tiles
-        out[ok, :, :, h, :] = chunks[t[ok]][:, :, np.arange(16) % 4, :]
+    ks = (kc + 3) // 4
+    chunks = sf.reshape(-1)[: tiles * kc * 512].reshape(tiles, kc, 512)   # [tile, k, 512]
+    out = np.zeros((nb, ks, 2, 4, 512), dtype=np.uint8)
+    for blk in range(nb):
+        for h in range(2):
+            t = 2 * blk + h
+            if t >= tiles:
+                continue
+            for k in range(kc):
+                out[blk, k // 4, h, k % 4] = chunks[t, k]
     return out.reshape(-1)
 
 
