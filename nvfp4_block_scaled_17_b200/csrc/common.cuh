@@ -315,69 +315,12 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] x B[smem]^T with per-16 E4M3 block scales from tensor memory.
-__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{\n\t"
-        ".reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
-        "[%6], p;\n\t"
-        "}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-        : "memory");
-}
-
-// D[tmem] (+)= A x B^T on signed int8 operands with an int32 accumulator (kind::i8; no
-// scale factors).
-__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t"
-        ".reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t"
-        "}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrive on `bar` once every tcgen05 operation issued so far by this thread is done.
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-
-// 32 lanes x 128 bits from shared memory, broadcast to all four lane quadrants.
-__device__ __forceinline__ void tc_copy_sf(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
-}
-
-// Warp-issued forms of the MMA, copy and commit above: the whole warp executes the call,
-// converged, and elect.sync lets one lane (the lowest, the same one every time, so its
-// commits track all of its operations) issue the operation.  Keeping the issuing loop
-// warp-uniform lets the compiler hold descriptors, addresses and counters in uniform
-// registers; a loop run by a single lane of the warp issued the same operations at well
-// under half the tensor-pipe rate.
-__device__ __forceinline__ void mma_nvf4_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                           uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                           uint32_t accumulate) {
-    asm volatile(
-        "{\n\t"
-        ".reg .pred p, e;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
-        "[%6], p;\n\t"
-        "}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-        : "memory");
-}
+// Warp-issued tcgen05 operations: the whole warp executes the call, converged, and
+// elect.sync lets one lane (the lowest, the same one every time, so its commits track all
+// of its operations) issue the operation.  The issuing loops stay warp-uniform, which
+// lets the compiler hold descriptors, addresses and counters in uniform registers; the
+// same operations issued from a loop run by a single lane of the warp reached the tensor
+// pipe at 0.65x the rate.
 __device__ __forceinline__ void mma_i8_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -396,11 +339,6 @@ __device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
         "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
             smem_u32(bar))
         : "memory");
-}
-__device__ __forceinline__ void tc_copy_sf_w(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-                 "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
 }
 
 // One K step of the block-scaled MMA, warp-issued with a single election: the step's

@@ -83,6 +83,57 @@ struct SmallParams {
     uint64_t budget_ns;
 };
 
+// One K step, warp-issued under a single election: the weight scales of row tile 0 (and,
+// with TWO, of row tile 1, 2048 bytes further) and the activation's into the slot's
+// columns 0, 4 and 8, then the M = 128 MMA of each row tile (row tile 1's W rows 16 KiB,
+// 1024 descriptor units, after tile 0's).
+template <bool TWO>
+__device__ __forceinline__ void small_step_w(uint32_t acc0, uint32_t acc1, uint64_t wd,
+                                             uint64_t xd, uint32_t idesc, uint32_t sf_t,
+                                             uint64_t sfw_d, uint64_t sfx_d,
+                                             uint32_t accumulate) {
+    if constexpr (TWO) {
+        asm volatile(
+            "{\n\t"
+            ".reg .pred p, e;\n\t"
+            ".reg .b32 t4, t8;\n\t"
+            ".reg .b64 s2, w1;\n\t"
+            "elect.sync _|e, 0xffffffff;\n\t"
+            "setp.ne.b32 p, %8, 0;\n\t"
+            "add.u32 t4, %5, 4;\n\t"
+            "add.u32 t8, %5, 8;\n\t"
+            "add.u64 s2, %6, 128;\n\t"
+            "add.u64 w1, %2, 1024;\n\t"
+            "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%5], %6;\n\t"
+            "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [t4], s2;\n\t"
+            "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [t8], %7;\n\t"
+            "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %2, %3, %4, "
+            "[%5], [t8], p;\n\t"
+            "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%1], w1, %3, %4, "
+            "[t4], [t8], p;\n\t"
+            "}" ::"r"(acc0),
+            "r"(acc1), "l"(wd), "l"(xd), "r"(idesc), "r"(sf_t), "l"(sfw_d), "l"(sfx_d),
+            "r"(accumulate)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t"
+            ".reg .pred p, e;\n\t"
+            ".reg .b32 t8;\n\t"
+            "elect.sync _|e, 0xffffffff;\n\t"
+            "setp.ne.b32 p, %8, 0;\n\t"
+            "add.u32 t8, %5, 8;\n\t"
+            "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%5], %6;\n\t"
+            "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [t8], %7;\n\t"
+            "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %2, %3, %4, "
+            "[%5], [t8], p;\n\t"
+            "}" ::"r"(acc0),
+            "r"(acc1), "l"(wd), "l"(xd), "r"(idesc), "r"(sf_t), "l"(sfw_d), "l"(sfx_d),
+            "r"(accumulate)
+            : "memory");
+    }
+}
+
 template <bool RSB, bool F32>
 __global__ void __launch_bounds__(XTHREADS, 1)
 gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -208,24 +259,27 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
                 }
                 tc_fence_after();
                 const int steps = min(4, p.kchunks - 4 * kt);
+                // the stage's descriptors; step kk adds 32 bytes to W and x (2 units) and
+                // 512 to the scale chunks (32 units).  Both weight scale layouts leave the
+                // stage's chunks in the same shared-memory order.
                 const uint32_t w0 = smem_u32(smem + stage * XS_STAGE);
-                const uint32_t x0 = w0 + XS_W;
-                const uint32_t sfw0 = x0 + XS_X;
-                const uint32_t sfx0 = sfw0 + XS_SFW;
-                for (int kk = 0; kk < steps; ++kk) {
-                    const uint32_t sf_t = tmem + XTMEM_SF + 12u * (uint32_t)slot;
-                    // both weight scale layouts leave the stage's chunks in the same order
-                    tc_copy_sf_w(sf_t, sdesc_sf(sfw0 + 512 * kk));
-                    if (two) tc_copy_sf_w(sf_t + 4, sdesc_sf(sfw0 + 2048 + 512 * kk));
-                    tc_copy_sf_w(sf_t + 8, sdesc_sf(sfx0 + 512 * kk));
-                    const uint64_t xdesc = sdesc_kmajor_sw128(x0 + 32 * kk);
-                    const uint32_t acc = (kt > kt_begin || kk > 0) ? 1u : 0u;
-                    mma_nvf4_w(tmem, sdesc_kmajor_sw128(w0 + 32 * kk), xdesc, p.idesc, sf_t,
-                               sf_t + 8, acc);
-                    if (two)
-                        mma_nvf4_w(tmem + XTMEM_ACC1, sdesc_kmajor_sw128(w0 + 16384 + 32 * kk),
-                                   xdesc, p.idesc, sf_t + 4, sf_t + 8, acc);
-                    if (++slot == XSF_SLOTS) slot = 0;
+                const uint64_t wd = sdesc_kmajor_sw128(w0);
+                const uint64_t xd = sdesc_kmajor_sw128(w0 + XS_W);
+                const uint64_t sfw_d = sdesc_sf(w0 + XS_W + XS_X);
+                const uint64_t sfx_d = sdesc_sf(w0 + XS_W + XS_X + XS_SFW);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    if (kk < steps) {
+                        const uint32_t sf_t = tmem + XTMEM_SF + 12u * (uint32_t)slot;
+                        const uint32_t acc = (kt > kt_begin || kk > 0) ? 1u : 0u;
+                        if (two)
+                            small_step_w<true>(tmem, tmem + XTMEM_ACC1, wd + 2 * kk, xd + 2 * kk,
+                                               p.idesc, sf_t, sfw_d + 32 * kk, sfx_d + 32 * kk, acc);
+                        else
+                            small_step_w<false>(tmem, tmem + XTMEM_ACC1, wd + 2 * kk, xd + 2 * kk,
+                                                p.idesc, sf_t, sfw_d + 32 * kk, sfx_d + 32 * kk, acc);
+                        slot = slot == XSF_SLOTS - 1 ? 0 : slot + 1;
+                    }
                 }
                 tc_commit_w(&empty[stage]);
                 if (++stage == XSTAGES) {
