@@ -178,13 +178,14 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
     auto load_w = [&](int stage, int kt, int steps) {
         uint8_t* sW = smem + stage * XS_STAGE;
         uint8_t* sSFW = sW + XS_W + XS_X;
-        tma_load_2d(sW, &tmW, &full[stage], kt * XBKB, tile * XW_ROWS);
+        tma_load_2d_w(sW, &tmW, &full[stage], kt * XBKB, tile * XW_ROWS);
         if constexpr (RSB) {
-            bulk_load(sSFW, p.sfw + ((size_t)tile * p.k_tiles + kt) * 4096, 4096u, &full[stage]);
+            bulk_load_w(sSFW, p.sfw + ((size_t)tile * p.k_tiles + kt) * 4096, 4096u, &full[stage]);
         } else {
             for (int t = 0; t < (two ? 2 : 1); ++t)
-                bulk_load(sSFW + t * 2048, p.sfw + ((size_t)(2 * tile + t) * p.kchunks + 4 * kt) * 512,
-                          (uint32_t)steps * 512u, &full[stage]);
+                bulk_load_w(sSFW + t * 2048,
+                            p.sfw + ((size_t)(2 * tile + t) * p.kchunks + 4 * kt) * 512,
+                            (uint32_t)steps * 512u, &full[stage]);
         }
     };
     auto stage_bytes = [&](int steps) -> uint32_t {
@@ -195,16 +196,19 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
     // With w_early the weight copies of the first stages go out before the wait for the
     // previous kernel (which wrote the activation, not the weights); the activation's
     // copies follow the wait.
+    // Warp 0 issues its copies converged, one elected lane per copy (the _w forms).
     int n_early = 0;
-    if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmW);
-        prefetch_tensormap(&tmX);
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tensormap(&tmW);
+            prefetch_tensormap(&tmX);
+        }
         if (p.w_early) {
             n_early = min(XSTAGES, kt_end - kt_begin);
             for (int i = 0; i < n_early; ++i) {
                 const int kt = kt_begin + i;
                 const int steps = min(4, p.kchunks - 4 * kt);
-                mbar_arrive_expect_tx(&full[i], stage_bytes(steps));
+                mbar_arrive_expect_tx_w(&full[i], stage_bytes(steps));
                 load_w(i, kt, steps);
             }
         }
@@ -213,24 +217,24 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
     griddep_launch_dependents();
 
     if (warp == 0) {
-        if (lane == 0) {
+        {
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, issued_phase = 0;
             for (int kt = kt_begin; kt < kt_end; ++kt) {
                 const int steps = min(4, p.kchunks - 4 * kt);
                 if (kt - kt_begin >= n_early) {
-                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status,
-                                           p.budget_ns))
+                    if (!mbar_wait_bounded_warp(&empty[stage], phase ^ 1, abort_flag, p.status,
+                                                p.budget_ns))
                         break;
-                    mbar_arrive_expect_tx(&full[stage], stage_bytes(steps));
+                    mbar_arrive_expect_tx_w(&full[stage], stage_bytes(steps));
                     load_w(stage, kt, steps);
                 }
                 uint8_t* sX = smem + stage * XS_STAGE + XS_W;
                 uint8_t* sSFX = sX + XS_X + XS_SFW;
                 const uint32_t sfx_bytes = (uint32_t)steps * 512u;
-                tma_load_2d(sX, &tmX, &full[stage], kt * XBKB, 0);
-                bulk_load(sSFX, p.sfx + (size_t)(4 * kt) * 512, sfx_bytes, &full[stage]);
+                tma_load_2d_w(sX, &tmX, &full[stage], kt * XBKB, 0);
+                bulk_load_w(sSFX, p.sfx + (size_t)(4 * kt) * 512, sfx_bytes, &full[stage]);
                 issued |= 1u << stage;
                 issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                 if (++stage == XSTAGES) {
@@ -238,7 +242,7 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant
                     phase ^= 1;
                 }
             }
-            // every fill this thread started must land before the block can exit
+            // every fill this warp started must land before the block can exit
             for (int s = 0; s < XSTAGES; ++s)
                 if (issued & (1u << s)) {
                     volatile int no_abort = 0;
