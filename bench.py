@@ -622,6 +622,39 @@ def leg_gemm_m_sweep(dev, pk, l2):
                         "alone (eager_us: events around each eager call)", "points": points}
 
 
+def leg_gemm_square(dev, pk, l2):
+    """The GEMM alone at 8192 x 8192 x 8192 (no bias), with 128x4 and with prepared weight
+    scales: each launch timed by events after a write of 256 MiB (more than L2).  Random
+    packed operands with finite E4M3 block scales (0.5 .. 0.94); 1.1 TFLOP per launch."""
+    M = N = K = 8192
+    g = torch.Generator(device=dev).manual_seed(1007)
+
+    def operand(rows):
+        packed = torch.randint(0, 256, (rows, K // 2), generator=g, device=dev,
+                               dtype=torch.int32).to(torch.uint8)
+        sf = (0x30 + torch.randint(0, 16, (nv.nvfp4_scale_bytes(rows, K),), generator=g,
+                                   device=dev, dtype=torch.int32)).to(torch.uint8)
+        return packed, sf
+
+    xp, xsf = operand(M)
+    wp, wsf = operand(N)
+    wsf_p = nv.prepare_weight_scales(wsf, N, K)
+    alpha = torch.tensor([1e-3], device=dev)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    flush = l2_flush_buffer(dev)
+    out = {"workload": "nvfp4_gemm / nvfp4_gemm_prepared at 8192^3, no bias, L2 flushed "
+                       "before each launch, 20 launches after 3 warm-up"}
+    for name, call in (
+            ("128x4", lambda: nv.nvfp4_gemm(xp, xsf, wp, wsf, alpha, None, M, N, K, out=y)),
+            ("prepared", lambda: nv.nvfp4_gemm_prepared(xp, xsf, wp, wsf_p, alpha, None, M, N,
+                                                        K, out=y))):
+        ms = time_each(call, 20, flush)
+        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        out[name] = {"us": ms * 1e3, "TFLOP/s": tf, "frac_of_fp4_peak": tf / pk["fp4"]}
+    del flush
+    return out
+
+
 def leg_weight_pack(dev, pk, l2):
     """Offline weight packing at the text-encoder scale: the seven Qwen3-VL projection
     shapes of one layer (487.6 M values, N(0, 0.02), generated untimed), each quantized with
@@ -799,6 +832,7 @@ LEGS = {
     "down_proj": leg_down_proj,
     "linear_m_sweep": leg_linear_m_sweep,
     "gemm_m_sweep": leg_gemm_m_sweep,
+    "gemm_square": leg_gemm_square,
     "weight_pack": leg_weight_pack,
     "dequant": leg_dequant,
     "fused_chain": leg_fused_chain,
